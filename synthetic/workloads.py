@@ -1,0 +1,178 @@
+"""Workload shapes and seeded input draws for video-DiT-shaped block-sparse attention.
+
+The five workloads mirror the sizes the LVSA, CalibAtt and SQuad pages talk about:
+Wan-2.1-like latent grids (21 frames of 30x52 or 45x80 latent tokens, 81 frames for
+long video), 12 or 40 heads of dimension 128, 128x128 blocks, and a tiny 256-token case
+that a pure-Python check finishes instantly.
+
+Everything here is deterministic from integer seeds, so the same tensors appear on any
+machine.  Nothing here computes attention, token order or masks from the method: the
+static "calibrated" mask below is a random input (the pages obtain such masks offline
+from model calibration, which needs trained weights).
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Iterable, List, Optional
+
+import numpy as np
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One video-shaped attention problem.
+
+    Tokens of the latent grid ``T x Hg x Wg`` are the sequence; ``tile`` is the 3D tile
+    (tt, th, tw) used to reorder them; ``block_size`` is the square attention block.
+    """
+
+    name: str
+    B: int
+    H: int
+    d: int
+    T: int
+    Hg: int
+    Wg: int
+    tile: tuple
+    block_size: int
+    seed: int
+    k_offset: float = 0.0
+
+    @property
+    def n_valid(self) -> int:
+        return self.T * self.Hg * self.Wg
+
+    @property
+    def n_pad(self) -> int:
+        bs = self.block_size
+        return (self.n_valid + bs - 1) // bs * bs
+
+    @property
+    def nb(self) -> int:
+        return self.n_pad // self.block_size
+
+    @property
+    def frame_tokens(self) -> int:
+        return self.Hg * self.Wg
+
+    @property
+    def scale(self) -> float:
+        # float32 value of 1/sqrt(d); both sides use exactly this float.
+        return float(np.float32(1.0 / math.sqrt(self.d)))
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", B=1, H=2, d=64, T=4, Hg=8, Wg=8, tile=(1, 4, 4),
+                     block_size=64, seed=0),
+    "small": Workload("small", B=1, H=12, d=128, T=21, Hg=30, Wg=52, tile=(1, 8, 16),
+                      block_size=128, seed=1),
+    "static": Workload("static", B=1, H=12, d=128, T=21, Hg=30, Wg=52, tile=(1, 8, 16),
+                       block_size=128, seed=2),
+    "large": Workload("large", B=1, H=40, d=128, T=21, Hg=45, Wg=80, tile=(1, 8, 16),
+                      block_size=128, seed=3, k_offset=0.5),
+    "long": Workload("long", B=1, H=12, d=128, T=81, Hg=30, Wg=52, tile=(1, 8, 16),
+                     block_size=128, seed=4),
+}
+
+
+def _head_generator(seed: int, tensor: int, b: int, h: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(((seed * 1_000_003 + tensor * 10_007 + b * 101) * 1009 + h) % (2**62))
+    return g
+
+
+def make_qkv(w: Workload, heads: Optional[Iterable[int]] = None, dtype=torch.bfloat16):
+    """Draw raster-order Q, K, V of shape [B, H, n_valid, d] (bf16, round-to-nearest-even).
+
+    Each (tensor, b, h) slice has its own seeded generator, so any subset of heads can be
+    drawn alone and matches the full draw.  Values are iid N(0,1) in fp32 before the cast;
+    K gets ``w.k_offset`` added to every component (the same vector for all tokens of a
+    head) when the workload asks for it.
+    """
+    hs = list(range(w.H)) if heads is None else list(heads)
+    out = []
+    for t in range(3):
+        x = torch.empty((w.B, len(hs), w.n_valid, w.d), dtype=dtype)
+        for b in range(w.B):
+            for hi, h in enumerate(hs):
+                g = _head_generator(w.seed, t, b, h)
+                v = torch.randn((w.n_valid, w.d), generator=g, dtype=torch.float32)
+                if t == 1 and w.k_offset != 0.0:
+                    v += w.k_offset
+                x[b, hi] = v.to(dtype)
+        out.append(x)
+    return tuple(out)
+
+
+def static_calibrated_mask(w: Workload, density: float = 0.30, seed_base: int = 1000) -> np.ndarray:
+    """Random per-head static block mask [H, nb, nb] (uint8) standing in for a calibrated mask.
+
+    Blocks sit on a coarse spatiotemporal coordinate: ``u = (i + 0.5) * Bs / frame_tokens``
+    frames, split into a frame coordinate ``u`` and an in-frame coordinate ``frac(u)``.
+    Off-diagonal blocks are kept with probability ``min(1, c_h * exp(-dist / tau_h))``, where
+    ``tau_h`` varies by head and ``c_h`` is found by bisection so that the expected density,
+    counting the always-kept diagonal as 1, equals ``density``.  Draws come from numpy's
+    PCG64 seeded with ``seed_base + h``.
+    """
+    nb = w.nb
+    u = (np.arange(nb, dtype=np.float64) + 0.5) * w.block_size / w.frame_tokens
+    frac = u - np.floor(u)
+    dt = u[:, None] - u[None, :]
+    ds = 4.0 * (frac[:, None] - frac[None, :])
+    dist = np.sqrt(dt * dt + ds * ds)
+    eye = np.eye(nb, dtype=bool)
+    masks = np.zeros((w.H, nb, nb), dtype=np.uint8)
+    for h in range(w.H):
+        tau = 1.0 + 2.0 * h / max(1, w.H - 1)
+        base = np.exp(-dist / tau)
+
+        def expected(c):
+            p = np.minimum(1.0, c * base)
+            p[eye] = 1.0
+            return p.mean()
+
+        lo, hi = 0.0, 1.0
+        while expected(hi) < density:
+            hi *= 2.0
+        for _ in range(100):
+            mid = 0.5 * (lo + hi)
+            if expected(mid) < density:
+                lo = mid
+            else:
+                hi = mid
+        p = np.minimum(1.0, hi * base)
+        rng = np.random.default_rng(seed_base + h)
+        draw = rng.random((nb, nb))
+        masks[h] = ((draw < p) | eye).astype(np.uint8)
+    return masks
+
+
+def mask_variants(w: Workload) -> List[dict]:
+    """The block-mask specifications each workload is checked and measured with.
+
+    ``window_anchor`` entries give (unit tokens, radius in units, anchors, steps);
+    ``static`` entries carry a dense per-head mask; ``two_stage`` gives the window group
+    size in blocks; ``all`` is the dense mask.
+    """
+    if w.name == "tiny":
+        return [dict(label="win1_anchor1", kind="window_anchor", unit=w.block_size, radius=1,
+                     anchors=1, steps=[0])]
+    if w.name == "small":
+        return [dict(label="frame1_anchor4", kind="window_anchor", unit=w.frame_tokens,
+                     radius=1, anchors=4, steps=list(range(50)))]
+    if w.name == "static":
+        return [dict(label="static30", kind="static", density=0.30),
+                dict(label="all", kind="all")]
+    if w.name == "large":
+        return [dict(label=f"band{r}_anchor4", kind="window_anchor", unit=w.block_size,
+                     radius=r, anchors=4, steps=[0]) for r in (28, 60, 171)]
+    if w.name == "long":
+        # Window groups of about sqrt(n) tokens: round(sqrt(n_pad) / Bs) blocks.
+        g = int(round(math.sqrt(w.n_pad) / w.block_size))
+        return ([dict(label="two_stage", kind="two_stage", group=g)]
+                + [dict(label=f"band{r}_anchor4", kind="window_anchor", unit=w.block_size,
+                        radius=r, anchors=4, steps=[0]) for r in (23, 48, 130, 287)]
+                + [dict(label="all", kind="all")])
+    raise KeyError(w.name)
