@@ -1,0 +1,372 @@
+"""Benchmark: block-sparse attention layer path on B200, one JSON line on rank 0.
+
+A step is one pass of the whole hot path over one layer of the video-DiT-small-like
+workload (B=1 per GPU, 12 heads, head dim 128, latent grid 21x30x52 = 32,760 tokens padded to
+32,768, 1x8x16 tiles, 128x128 blocks, +-1 latent-frame window + 4 rotating anchor blocks):
+tile reorder of Q, K and V, CSR build for denoising step s = k mod 50, block-sparse
+attention, inverse reorder of O.  Inputs (302 MB of Q/K/V, larger than the 126 MB L2) are
+resident in HBM before the timed region.
+
+  value      effective TFLOP/s over active blocks (4*Bs^2*d per active block pair and head)
+             for the whole step, summed over ranks, divided by the max-over-ranks time.
+  roofline   the attention kernel alone (CUDA events on its launch stream).
+  e2e        the same metric through the public API with pinned host buffers: H2D of
+             Q/K/V and D2H of O and LSE inside the timed region.
+  cpu_baseline  the FP64 oracle on a bounded, time-limited sample of the same workload.
+
+``--impl reference`` times the oracle itself as the reference arm (rank 0 only).
+Multi-GPU (torchrun): every rank runs its own batch element (weak scaling, no collective
+on the data path; a barrier and a max-reduce of the timings only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from synthetic import WORKLOADS, Workload, make_qkv, mask_variants  # noqa: E402
+
+METRIC = "block-sparse attn effective TFLOP/s (active blocks) & % bf16 TC peak; ms/layer"
+WORKLOAD = "small"
+ATTN_SRC = os.path.join(ROOT, "block_sparse_attention_lva_b200", "csrc", "attn.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "bsa_fwd_small_traffic.json")
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _workload_for_rank(rank: int) -> Workload:
+    w = WORKLOADS[WORKLOAD]
+    return Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+
+
+def _config_dict(w: Workload, spec: dict, n_gpus: int) -> dict:
+    return {"workload": f"video-DiT-small-like: B=1 per GPU, {w.H} heads, d={w.d}, latent grid "
+                        f"{w.T}x{w.Hg}x{w.Wg}={w.n_valid} tokens padded to {w.n_pad}, tiles 1x8x16, "
+                        f"{w.block_size}x{w.block_size} blocks, +-1 latent-frame window + 4 rotating "
+                        f"anchor blocks, denoising step = step index mod 50",
+            "global_batch": n_gpus * w.B, "heads": w.H, "head_dim": w.d, "seq_len": w.n_pad,
+            "block": w.block_size, "step_contents": "3x reorder + CSR build + attention + inverse reorder",
+            "l2": "inputs larger than L2 (302 MB Q/K/V per GPU), no flush",
+            "parallelism": f"dp{n_gpus} (independent batch elements)"}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("bf16_tflops"), d.get("bf16_tflops_sustained"), d.get("hbm_gbs"), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _traffic_per_launch():
+    """DRAM bytes per attention launch from the committed ncu summary, if it matches the source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
+    return d.get("bytes_per_launch") if d.get("attn_cu_sha256") == sha else None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _flops_per_nnz(w: Workload) -> float:
+    return 4.0 * w.block_size * w.block_size * w.d
+
+
+def _nnz_table(layer, steps):
+    """Active block pairs of the mask at each denoising step (read back outside timing)."""
+    table = {}
+    for s in steps:
+        layer.build_mask(s)
+        table[s] = int(layer.nnz.item())
+    return table
+
+
+def run_lva(args):
+    import torch.distributed as dist
+
+    import block_sparse_attention_lva_b200 as lva
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    w = _workload_for_rank(rank)
+    spec = mask_variants(WORKLOADS[WORKLOAD])[0]
+    n_steps_cycle = len(spec["steps"])
+    q, k, v = make_qkv(w)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    layer = lva.VideoBlockSparseAttention(w.B, w.H, w.d, (w.T, w.Hg, w.Wg), w.tile, w.block_size, spec,
+                                          scale=w.scale, device=dev)
+    nnz = _nnz_table(layer, range(n_steps_cycle))
+    fpn = _flops_per_nnz(w) * w.B * w.H          # mask_heads = 1: every head shares the CSR
+    stream = torch.cuda.current_stream(dev)
+
+    def step(kidx, ev=None):
+        s = kidx % n_steps_cycle
+        layer.reorder_in(qd, kd, vd)
+        layer.build_mask(s)
+        if ev is not None:
+            ev[0].record(stream)
+        layer.attend()
+        if ev is not None:
+            ev[1].record(stream)
+        layer.reorder_out()
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    for kk in range(args.warmup):
+        step(kk)
+    torch.cuda.synchronize()
+    status, detail = lva.lva_device_error()
+    if status != 0:
+        raise RuntimeError(f"kernel error word {status} ({detail}) during warm-up")
+
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    base = args.warmup
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for kk in range(args.steps):
+            step(base + kk, attn_ev[kk])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms_total = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
+    flops = sum(nnz[(base + kk) % n_steps_cycle] for kk in range(args.steps)) * fpn
+    status, detail = lva.lva_device_error()
+    if status != 0:
+        raise RuntimeError(f"kernel error word {status} ({detail}) during timing")
+
+    # ---------------- e2e through the public API with pinned host buffers
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty((w.B, w.H, w.n_valid, w.d), dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty((w.B, w.H, w.n_pad), dtype=torch.float32).pin_memory()
+    qe, ke, ve = (torch.empty_like(x) for x in (qd, kd, vd))
+
+    def e2e_step(kidx):
+        qe.copy_(qh, non_blocking=True)
+        ke.copy_(kh, non_blocking=True)
+        ve.copy_(vh, non_blocking=True)
+        o, lse = layer(qe, ke, ve, step=kidx % n_steps_cycle)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    for kk in range(args.warmup):
+        e2e_step(kk)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for kk in range(args.steps):
+        e2e_step(base + kk)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+    h2d = 3 * qh.numel() * qh.element_size()
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    # ---------------- reduce over ranks (max time, summed work)
+    times = torch.tensor([ms_total, ms_e2e, float(np.mean(attn_ms))], dtype=torch.float64, device=dev)
+    work = torch.tensor([flops], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(times, op=dist.ReduceOp.MAX)
+        dist.all_reduce(work, op=dist.ReduceOp.SUM)
+    ms_total, ms_e2e, attn_ms_mean = times.tolist()
+    flops_all = work.item()
+
+    if rank == 0:
+        burst, sustained, hbm, peak_kind = _peaks()
+        attn_flops_launch = flops / args.steps                   # this rank's mean per launch
+        achieved = attn_flops_launch / (attn_ms_mean * 1e-3) / 1e12
+        traffic = _traffic_per_launch()
+        line = {
+            "metric": METRIC, "value": flops_all / (ms_total * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q/K/V)",
+            "config": _config_dict(w, spec, ws),
+            "attn_ms_per_layer": attn_ms_mean,
+            "active_block_pairs_per_head": {"min": min(nnz.values()), "max": max(nnz.values()),
+                                             "density": float(np.mean(list(nnz.values()))) / w.nb ** 2},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                         "frac": achieved / sustained, "traffic": traffic,
+                         "peak_kind": f"{peak_kind} bf16 dense, sustained (kernel timed inside back-to-back steps)",
+                         "frac_of_burst": achieved / burst, "kernel": "bsa_fwd_kernel<128,128>"},
+            "clocks": clocks.summary(),
+            "e2e": {"value": flops_all / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": ms_e2e / args.steps},
+            "gpu_launches": 8 * args.steps,
+        }
+        if ws == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(w, spec, args.cpu_seconds)
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+
+
+def _oracle_sample(w, spec, q, k, v, perm, seconds, seed):
+    """Runs the oracle on seeded random (head, query block) items until `seconds` pass."""
+    from oracle.attention import attention_blocked
+    from oracle.mask import window_anchor_mask
+    from oracle.reorder import reorder_forward
+
+    rng = np.random.default_rng(seed)
+    P = w.B * w.H
+    tile = [torch.from_numpy(reorder_forward(x.view(torch.int16).reshape(P, w.n_valid, w.d).numpy(), perm, w.n_pad))
+            .view(torch.bfloat16).reshape(w.B, w.H, w.n_pad, w.d) for x in (q, k, v)]
+    s = int(rng.integers(0, len(spec["steps"])))
+    m = window_anchor_mask(w.n_pad, w.n_valid, w.block_size, spec["unit"], spec["radius"], spec["anchors"], s)
+    flops, items = 0.0, 0
+    t0 = time.perf_counter()
+    while time.perf_counter() - t0 < seconds or items < 4:
+        h, i = int(rng.integers(0, w.H)), int(rng.integers(0, w.nb))
+        attention_blocked(tile[0][:, h:h + 1], tile[1][:, h:h + 1], tile[2][:, h:h + 1], m, w.block_size,
+                          w.n_valid, w.scale, query_blocks=[(0, 0, i)])
+        flops += int(m[i].sum()) * _flops_per_nnz(w)
+        items += 1
+    return flops, time.perf_counter() - t0, items
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, spec, seconds):
+    from oracle.reorder import tile_permutation
+    q, k, v = make_qkv(w)
+    perm = tile_permutation(w.T, w.Hg, w.Wg, *w.tile)
+    flops, secs, items = _oracle_sample(w, spec, q, k, v, perm, seconds, seed=7)
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+            "sample": f"{items} random (head, query block) items of the same workload (one denoising step's "
+                      f"mask), {secs:.1f} s of FP64 numpy/BLAS work; the whole step is attention-dominated"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return
+    from oracle.reorder import tile_permutation
+    w = _workload_for_rank(0)
+    spec = mask_variants(WORKLOADS[WORKLOAD])[0]
+    q, k, v = make_qkv(w)
+    perm = tile_permutation(w.T, w.Hg, w.Wg, *w.tile)
+    per_step = args.reference_seconds
+    for kk in range(args.warmup):
+        _oracle_sample(w, spec, q, k, v, perm, per_step / 4, seed=100 + kk)
+    tot_f, tot_s, tot_items = 0.0, 0.0, 0
+    for kk in range(args.steps):
+        f, s, n = _oracle_sample(w, spec, q, k, v, perm, per_step, seed=kk)
+        tot_f, tot_s, tot_items = tot_f + f, tot_s + s, tot_items + n
+    value = tot_f / tot_s / 1e12
+    sample = (f"each step: random (head, query block) items of the same workload for ~{per_step:.0f} s "
+              f"({tot_items} items over {args.steps} steps)")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_s / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) bf16 Q/K/V)", "config": _config_dict(w, spec, ws),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": _threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lva", choices=["lva", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=5.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_lva(args)
+
+
+if __name__ == "__main__":
+    main()

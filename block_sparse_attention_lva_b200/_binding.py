@@ -1,0 +1,192 @@
+"""ctypes binding of ``liblva.so`` (the C ABI of ``include/lva.h``).
+
+Argument marshalling only: each function takes torch tensors that live on the current
+CUDA device, passes their device pointers and the current stream to the C function of the
+same name, and raises ``LvaError`` on a non-OK status.  All computation happens in the
+library's CUDA kernels; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblva.so")
+
+LVA_OK = 0
+LVA_MASK_WINDOW_ANCHOR = 0
+LVA_MASK_STATIC = 1
+LVA_MASK_ALL = 2
+LVA_MASK_TWO_STAGE = 3
+
+STATUS_NAMES = {0: "LVA_OK", 1: "LVA_ERR_INVALID_ARG", 2: "LVA_ERR_UNSUPPORTED",
+                3: "LVA_ERR_CAPACITY", 4: "LVA_ERR_CUDA", 5: "LVA_ERR_TIMEOUT"}
+
+# Every symbol the header declares, with its ctypes signature.
+_c_i64, _c_int, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+
+
+class LvaMaskParams(ctypes.Structure):
+    """Mirror of ``lva_mask_params``."""
+    _fields_ = [("kind", ctypes.c_int), ("mask_heads", ctypes.c_int), ("block_size", ctypes.c_int),
+                ("n_pad", ctypes.c_int64), ("n_valid", ctypes.c_int64),
+                ("window_unit_tokens", ctypes.c_int64), ("window_radius", ctypes.c_int),
+                ("num_anchors", ctypes.c_int), ("step", ctypes.c_int), ("group_blocks", ctypes.c_int)]
+
+
+SIGNATURES = {
+    "lva_status_string": (ctypes.c_char_p, [_c_int]),
+    "lva_last_error_message": (ctypes.c_char_p, []),
+    "lva_version": (_c_int, []),
+    "lva_reorder_tokens": (_c_int, [_vp, _vp, _c_i64, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                    _c_i64, _c_i64, _c_int, _c_int, _vp]),
+    "lva_block_mask_max_nnz": (_c_i64, [ctypes.POINTER(LvaMaskParams)]),
+    "lva_build_block_mask": (_c_int, [ctypes.POINTER(LvaMaskParams), _vp, _vp, _vp, _c_i64, _vp, _vp]),
+    "lva_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
+                                       _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp]),
+    "lva_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+}
+
+
+class LvaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build the CUDA library first "
+            "(python -c 'import __graft_entry__ as g; g.build()' or python block_sparse_attention_lva_b200/build.py)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int):
+    if status != LVA_OK:
+        raise LvaError(status, lib.lva_last_error_message().decode())
+
+
+def _stream(device=None) -> int:
+    import torch
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _need(cond: bool, msg: str):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _cuda_tensor(t, name: str, dtype=None, numel: int = None):
+    """Checks that ``t`` is a contiguous CUDA tensor (of ``dtype``, with >= ``numel`` elements)."""
+    _need(t is not None and t.is_cuda, f"{name} must be a CUDA tensor")
+    _need(t.is_contiguous(), f"{name} must be contiguous")
+    if dtype is not None:
+        _need(t.dtype == dtype, f"{name} must be {dtype}, got {t.dtype}")
+    if numel is not None:
+        _need(t.numel() >= numel, f"{name} has {t.numel()} elements, needs {numel}")
+
+
+@dataclass
+class MaskParams:
+    """Python view of ``lva_mask_params``."""
+    kind: int
+    n_pad: int
+    n_valid: int
+    block_size: int = 128
+    mask_heads: int = 1
+    window_unit_tokens: int = 1
+    window_radius: int = 0
+    num_anchors: int = 0
+    step: int = 0
+    group_blocks: int = 1
+
+    def to_c(self) -> LvaMaskParams:
+        return LvaMaskParams(self.kind, self.mask_heads, self.block_size, self.n_pad, self.n_valid,
+                             self.window_unit_tokens, self.window_radius, self.num_anchors, self.step,
+                             self.group_blocks)
+
+
+def lva_version() -> int:
+    return lib.lva_version()
+
+
+def lva_reorder_tokens(src, dst, grid, tile, n_pad: int, inverse: bool = False):
+    """Tile-order gather (``inverse=False``: src [P, N, row] -> dst [P, n_pad, row]) or the
+    inverse scatter (src [P, n_pad, row] -> dst [P, N, row]); rows are the trailing dims."""
+    T, H, W = grid
+    n = T * H * W
+    planes = src.shape[0]
+    row_elems = 1
+    for x in src.shape[2:]:
+        row_elems *= x
+    _cuda_tensor(src, "src", numel=planes * (n_pad if inverse else n) * row_elems)
+    _cuda_tensor(dst, "dst", dtype=src.dtype, numel=planes * (n if inverse else n_pad) * row_elems)
+    _need(src.shape[1] == (n_pad if inverse else n), "src rows must be n_pad (inverse) or T*H*W")
+    _check(lib.lva_reorder_tokens(_ptr(src), _ptr(dst), planes, T, H, W, tile[0], tile[1], tile[2],
+                                  n_pad, row_elems, src.element_size(), int(bool(inverse)),
+                                  ctypes.c_void_p(_stream(src.device))))
+    return dst
+
+
+def lva_block_mask_max_nnz(params: MaskParams) -> int:
+    cp = params.to_c()
+    return lib.lva_block_mask_max_nnz(ctypes.byref(cp))
+
+
+def lva_build_block_mask(params: MaskParams, dense_mask, row_ptr, col_idx, nnz_out):
+    """Build the CSR of a block mask on the GPU into caller-owned int32 buffers."""
+    import torch
+    nb = params.n_pad // params.block_size
+    _cuda_tensor(row_ptr, "row_ptr", torch.int32, params.mask_heads * nb + 1)
+    _cuda_tensor(col_idx, "col_idx", torch.int32)
+    _cuda_tensor(nnz_out, "nnz_out", torch.int32, 1)
+    if params.kind == LVA_MASK_STATIC:
+        _cuda_tensor(dense_mask, "dense_mask", torch.uint8, params.mask_heads * nb * nb)
+    else:
+        dense_mask = None
+    cp = params.to_c()
+    _check(lib.lva_build_block_mask(ctypes.byref(cp), _ptr(dense_mask), _ptr(row_ptr), _ptr(col_idx),
+                                    col_idx.numel(), _ptr(nnz_out),
+                                    ctypes.c_void_p(_stream(row_ptr.device))))
+    return row_ptr, col_idx, nnz_out
+
+
+def lva_block_sparse_attn(q, k, v, o, lse, n_valid: int, block_size: int, row_ptr, col_idx,
+                          mask_heads: int, scale: float):
+    """O, LSE of block-sparse softmax attention over the CSR-listed key blocks."""
+    import torch
+    B, H, n_pad, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _cuda_tensor(t, name, torch.bfloat16)
+        _need(tuple(t.shape) == (B, H, n_pad, d), f"{name} must have shape {(B, H, n_pad, d)}")
+    _cuda_tensor(lse, "lse", torch.float32, B * H * n_pad)
+    nb = n_pad // block_size
+    _cuda_tensor(row_ptr, "row_ptr", torch.int32, mask_heads * nb + 1)
+    _cuda_tensor(col_idx, "col_idx", torch.int32)
+    _check(lib.lva_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, n_pad, n_valid,
+                                     d, block_size, _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                                     mask_heads, ctypes.c_float(scale),
+                                     ctypes.c_void_p(_stream(q.device))))
+    return o, lse
+
+
+def lva_device_error(stream=None):
+    """(status, detail) of the kernel error word of the current device; clears it."""
+    st, det = ctypes.c_int(0), ctypes.c_int(0)
+    s = _stream() if stream is None else stream
+    _check(lib.lva_device_error(ctypes.c_void_p(s), ctypes.byref(st), ctypes.byref(det)))
+    return st.value, det.value

@@ -1,0 +1,216 @@
+// api.cu -- the C ABI declared in include/lva.h: argument checks, status codes, the
+// per-thread error message, the per-device kernel error word, and dispatch to launchers.
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include "kernels.h"
+#include "lva.h"
+
+namespace lva {
+namespace {
+
+thread_local char g_msg[256] = "";
+
+lva_status fail(lva_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+lva_status ok() {
+  g_msg[0] = '\0';
+  return LVA_OK;
+}
+
+lva_status from_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(LVA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// Kernel-side error word: [0] = status, [1] = detail.  One copy per device (module global);
+// its device address is looked up once per device.
+__device__ int g_device_error[2];
+
+int* g_err_ptr[128] = {};
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  if (g_err_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+}  // namespace lva
+
+using namespace lva;
+
+extern "C" {
+
+const char* lva_status_string(lva_status s) {
+  switch (s) {
+    case LVA_OK: return "LVA_OK";
+    case LVA_ERR_INVALID_ARG: return "LVA_ERR_INVALID_ARG";
+    case LVA_ERR_UNSUPPORTED: return "LVA_ERR_UNSUPPORTED";
+    case LVA_ERR_CAPACITY: return "LVA_ERR_CAPACITY";
+    case LVA_ERR_CUDA: return "LVA_ERR_CUDA";
+    case LVA_ERR_TIMEOUT: return "LVA_ERR_TIMEOUT";
+  }
+  return "LVA_ERR_UNKNOWN";
+}
+
+const char* lva_last_error_message(void) { return g_msg; }
+
+int lva_version(void) { return LVA_VERSION; }
+
+lva_status lva_reorder_tokens(const void* src, void* dst, int64_t planes, int T, int H, int W,
+                              int tile_t, int tile_h, int tile_w, int64_t n_pad, int64_t row_elems,
+                              int elem_bytes, int inverse, cudaStream_t stream) {
+  if (planes < 0) return fail(LVA_ERR_INVALID_ARG, "reorder: planes < 0");
+  if (T <= 0 || H <= 0 || W <= 0 || tile_t <= 0 || tile_h <= 0 || tile_w <= 0)
+    return fail(LVA_ERR_INVALID_ARG, "reorder: grid and tile sizes must be positive");
+  if (elem_bytes != 2 && elem_bytes != 4) return fail(LVA_ERR_INVALID_ARG, "reorder: elem_bytes must be 2 or 4");
+  if (row_elems <= 0) return fail(LVA_ERR_INVALID_ARG, "reorder: row_elems must be positive");
+  const int64_t n = int64_t(T) * H * W;
+  if (n >= (int64_t(1) << 31)) return fail(LVA_ERR_UNSUPPORTED, "reorder: T*H*W must be < 2^31");
+  if (n_pad < n || n_pad >= (int64_t(1) << 31)) return fail(LVA_ERR_INVALID_ARG, "reorder: need T*H*W <= n_pad < 2^31");
+  const int64_t row_bytes = row_elems * elem_bytes;
+  if (row_bytes > (int64_t(1) << 20)) return fail(LVA_ERR_UNSUPPORTED, "reorder: rows above 1 MiB");
+  if ((n_pad * row_bytes) / elem_bytes / 2 >= (int64_t(1) << 31) * 256)
+    return fail(LVA_ERR_UNSUPPORTED, "reorder: plane too large");
+  if (planes == 0) return ok();
+  if (src == nullptr || dst == nullptr) return fail(LVA_ERR_INVALID_ARG, "reorder: null pointer");
+  if (!aligned(src, elem_bytes) || !aligned(dst, elem_bytes))
+    return fail(LVA_ERR_INVALID_ARG, "reorder: pointers must be aligned to elem_bytes");
+  ReorderArgs a{src, dst, planes, T, H, W, tile_t, tile_h, tile_w, n, n_pad, row_bytes, inverse != 0};
+  return from_cuda(launch_reorder(a, stream), "reorder launch");
+}
+
+static lva_status check_mask_params(const lva_mask_params* p) {
+  if (p == nullptr) return fail(LVA_ERR_INVALID_ARG, "mask: null params");
+  if (p->block_size != 64 && p->block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "mask: block_size must be 64 or 128");
+  if (p->n_pad <= 0 || p->n_pad % p->block_size != 0) return fail(LVA_ERR_INVALID_ARG, "mask: n_pad must be a positive multiple of block_size");
+  if (p->n_valid < 1 || p->n_valid > p->n_pad) return fail(LVA_ERR_INVALID_ARG, "mask: need 1 <= n_valid <= n_pad");
+  if (p->mask_heads < 1) return fail(LVA_ERR_INVALID_ARG, "mask: mask_heads must be >= 1");
+  const int64_t nb = p->n_pad / p->block_size;
+  if (int64_t(p->mask_heads) * nb * nb >= (int64_t(1) << 31))
+    return fail(LVA_ERR_UNSUPPORTED, "mask: mask_heads*nb*nb must be < 2^31");
+  switch (p->kind) {
+    case LVA_MASK_WINDOW_ANCHOR:
+      if (p->window_unit_tokens < 1 || p->window_radius < 0 || p->num_anchors < 0 || p->step < 0)
+        return fail(LVA_ERR_INVALID_ARG, "mask: window needs unit >= 1, radius >= 0, anchors >= 0, step >= 0");
+      if (p->num_anchors > nb) return fail(LVA_ERR_INVALID_ARG, "mask: more anchors than blocks");
+      if (p->mask_heads != 1) return fail(LVA_ERR_INVALID_ARG, "mask: parametric kinds build one mask head");
+      break;
+    case LVA_MASK_TWO_STAGE:
+      if (p->group_blocks < 1) return fail(LVA_ERR_INVALID_ARG, "mask: group_blocks must be >= 1");
+      if (p->mask_heads != 1) return fail(LVA_ERR_INVALID_ARG, "mask: parametric kinds build one mask head");
+      break;
+    case LVA_MASK_ALL:
+      if (p->mask_heads != 1) return fail(LVA_ERR_INVALID_ARG, "mask: parametric kinds build one mask head");
+      break;
+    case LVA_MASK_STATIC:
+      break;
+    default:
+      return fail(LVA_ERR_INVALID_ARG, "mask: unknown kind %d", p->kind);
+  }
+  return ok();
+}
+
+int64_t lva_block_mask_max_nnz(const lva_mask_params* p) {
+  if (check_mask_params(p) != LVA_OK) return 0;
+  const int64_t nb = p->n_pad / p->block_size;
+  return int64_t(p->mask_heads) * nb * nb;
+}
+
+lva_status lva_build_block_mask(const lva_mask_params* p, const uint8_t* dense_mask, int32_t* row_ptr,
+                                int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
+                                cudaStream_t stream) {
+  lva_status s = check_mask_params(p);
+  if (s != LVA_OK) return s;
+  if (row_ptr == nullptr || col_idx == nullptr || nnz_out == nullptr)
+    return fail(LVA_ERR_INVALID_ARG, "mask: null output pointer");
+  if (!aligned(row_ptr, 4) || !aligned(col_idx, 4) || !aligned(nnz_out, 4))
+    return fail(LVA_ERR_INVALID_ARG, "mask: outputs must be 4-byte aligned");
+  if (p->kind == LVA_MASK_STATIC && dense_mask == nullptr)
+    return fail(LVA_ERR_INVALID_ARG, "mask: STATIC needs dense_mask");
+  const int64_t need = lva_block_mask_max_nnz(p);
+  if (col_capacity < need)
+    return fail(LVA_ERR_CAPACITY, "mask: col_capacity %lld < %lld", (long long)col_capacity, (long long)need);
+  MaskArgs a;
+  a.kind = p->kind;
+  a.mask_heads = p->mask_heads;
+  a.block_size = p->block_size;
+  a.n_pad = p->n_pad;
+  a.n_valid = p->n_valid;
+  a.unit_tokens = p->window_unit_tokens;
+  a.radius = p->window_radius;
+  a.num_anchors = p->num_anchors;
+  a.step = p->step;
+  a.group_blocks = p->group_blocks;
+  a.dense = dense_mask;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.nnz_out = nnz_out;
+  return from_cuda(launch_build_mask(a, stream), "mask launch");
+}
+
+lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int H, int64_t n_pad, int64_t n_valid, int d, int block_size,
+                                 const int32_t* row_ptr, const int32_t* col_idx, int64_t col_len,
+                                 int mask_heads, float scale, cudaStream_t stream) {
+  if (B < 0 || H < 1) return fail(LVA_ERR_INVALID_ARG, "attn: need B >= 0 and H >= 1");
+  if (d != 64 && d != 128) return fail(LVA_ERR_UNSUPPORTED, "attn: head dim must be 64 or 128");
+  if (block_size != 64 && block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "attn: block_size must be 64 or 128");
+  if (n_pad <= 0 || n_pad % block_size != 0) return fail(LVA_ERR_INVALID_ARG, "attn: n_pad must be a positive multiple of block_size");
+  if (n_valid < 0 || n_valid > n_pad) return fail(LVA_ERR_INVALID_ARG, "attn: need 0 <= n_valid <= n_pad");
+  if (mask_heads != 1 && mask_heads != H) return fail(LVA_ERR_INVALID_ARG, "attn: mask_heads must be 1 or H");
+  if (int64_t(B) * H * n_pad >= (int64_t(1) << 31)) return fail(LVA_ERR_UNSUPPORTED, "attn: B*H*n_pad must be < 2^31");
+  if (!(scale == scale)) return fail(LVA_ERR_INVALID_ARG, "attn: scale is NaN");
+  if (col_len < 0) return fail(LVA_ERR_INVALID_ARG, "attn: col_len < 0");
+  if (B == 0) return ok();
+  if (!q || !k || !v || !o || !lse || !row_ptr || (!col_idx && col_len > 0))
+    return fail(LVA_ERR_INVALID_ARG, "attn: null pointer");
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
+    return fail(LVA_ERR_INVALID_ARG, "attn: q, k, v, o must be 16-byte aligned");
+  if (!aligned(lse, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4))
+    return fail(LVA_ERR_INVALID_ARG, "attn: lse, row_ptr, col_idx must be 4-byte aligned");
+  int* err = device_error_word();
+  if (err == nullptr) return fail(LVA_ERR_CUDA, "attn: cannot locate the device error word");
+  AttnArgs a{q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr,
+             col_idx, col_len, mask_heads, scale, err};
+  const char* why = "launch";
+  cudaError_t e = launch_attn(a, stream, &why);
+  if (e != cudaSuccess) return fail(LVA_ERR_CUDA, "attn: %s: %s", why, cudaGetErrorString(e));
+  return ok();
+}
+
+lva_status lva_device_error(cudaStream_t stream, lva_status* status, int* detail) {
+  if (status == nullptr) return fail(LVA_ERR_INVALID_ARG, "device_error: null status");
+  int* err = device_error_word();
+  if (err == nullptr) return fail(LVA_ERR_CUDA, "device_error: cannot locate the device error word");
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return from_cuda(e, "device_error: stream sync");
+  int host[2] = {0, 0};
+  e = cudaMemcpy(host, err, sizeof(host), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return from_cuda(e, "device_error: read");
+  const int zero[2] = {0, 0};
+  e = cudaMemcpy(err, zero, sizeof(zero), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return from_cuda(e, "device_error: clear");
+  *status = static_cast<lva_status>(host[0]);
+  if (detail) *detail = host[1];
+  return ok();
+}
+
+}  // extern "C"

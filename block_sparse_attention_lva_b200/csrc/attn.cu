@@ -1,0 +1,418 @@
+// attn.cu -- block-sparse FlashAttention-style forward for sm_100a (TMA + tcgen05 + TMEM).
+//
+// One CTA computes one (batch, head, query block i): it walks only the key blocks listed
+// in CSR row (h_m, i) -- the precomputed skip list of the CalibAtt page ("Accelerating
+// Text-to-Video Generation with Calibrated Sparse Attention", section 2 B) or the LVSA
+// window + anchor set ("LVSA: Training-Free Sparse Attention for Long Video Diffusion",
+// technical summary section 2) -- with an online softmax, so the cost is proportional to
+// the number of listed blocks.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: Q tile once, then K_j / V_j tiles into a STAGES-deep ring;
+//   warp 1      MMA issuer (one thread): S = Q K_j^T into TMEM (two S buffers), and
+//               O += P V_j into a TMEM accumulator; owns the TMEM allocation;
+//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane = row): read S
+//               from TMEM, update running max / sum, write P (bf16) to shared memory in
+//               the tensor-core operand layout, rescale O in TMEM when the max moves by
+//               more than 2^8, and finally normalise O and write O and LSE.
+//
+// Shared-memory operands use the 128-byte swizzle that TMA writes: a 64-element (128 B)
+// slice of each row, eight rows per 1024-byte atom.  Q, K and P are K-major; V is read
+// MN-major straight from its [keys, d] layout.
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace lva {
+namespace {
+
+constexpr int BM = 128;            // query rows per MMA tile (TMEM lanes)
+constexpr int kThreads = 192;
+constexpr int kSoftmaxWarp0 = 2;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when max grows > 2^8
+constexpr uint32_t kTmemCols = 512;
+
+struct AttnParams {
+  int H, nb, mask_heads;
+  int64_t n_pad, n_valid;
+  float scale_log2;                // scale * log2(e)
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  int64_t col_len;
+  __nv_bfloat16* o;
+  float* lse;
+  int* err;
+};
+
+template <int D, int BN>
+struct Cfg {
+  static constexpr int STAGES = 2;
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full, o_done, final
+  static constexpr int NUM_BARS = 1 + 2 * STAGES + 2 + 2 + 1 + 1 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  // + slack for 1024-byte alignment; at least 120 KB so that one CTA (and one 512-column
+  // TMEM allocation) is resident per SM.
+  static constexpr int SMEM_RAW = OFF_MISC + 16 + 1024;
+  static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
+};
+
+// The CSR row of a work item, checked so that no read or TMA coordinate leaves its buffer.
+// Called by every thread (whole warps); each warp checks the row cooperatively, so every
+// role reaches the same answer from the same memory.
+__device__ __forceinline__ int csr_row(const AttnParams& p, int64_t row, int32_t& start,
+                                       bool& bad) {
+  const int32_t a = __ldg(p.row_ptr + row), b = __ldg(p.row_ptr + row + 1);
+  bad = !(a >= 0 && b >= a && int64_t(b) <= p.col_len);
+  start = 0;
+  if (bad) return 0;
+  bool lane_bad = false;
+  for (int32_t t = a + int32_t(threadIdx.x & 31); t < b; t += 32) {
+    const int32_t j = __ldg(p.col_idx + t);
+    lane_bad |= (j < 0 || j >= p.nb);
+  }
+  bad = __any_sync(0xffffffffu, lane_bad);
+  if (bad) return 0;
+  start = a;
+  return b - a;
+}
+
+template <int D, int BN>
+__global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = Cfg<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t sQ = s_base + C::OFF_Q, sK = s_base + C::OFF_K, sV = s_base + C::OFF_V,
+                 sP = s_base + C::OFF_P;
+  const uint32_t bar0 = s_base + C::OFF_BAR;
+  const uint32_t bar_q = bar0;
+  auto bar_kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+  auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + C::STAGES + s); };
+  auto bar_s_full = [&](int b) { return bar0 + 8u * (1 + 2 * C::STAGES + b); };
+  auto bar_s_free = [&](int b) { return bar0 + 8u * (3 + 2 * C::STAGES + b); };
+  const uint32_t bar_p_full = bar0 + 8u * (5 + 2 * C::STAGES);
+  const uint32_t bar_o_done = bar0 + 8u * (6 + 2 * C::STAGES);
+  const uint32_t bar_final = bar0 + 8u * (7 + 2 * C::STAGES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  // Stays zero: the drain waits after an abort are bounded by time alone.
+  volatile int* never = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Work item: plane-major, query block fastest, so neighbouring CTAs share one head's K/V.
+  const int64_t item = blockIdx.x;
+  const int64_t plane = item / p.nb;
+  const int i = int(item - plane * p.nb);
+  const int h = int(plane % p.H);
+  const int64_t csr = int64_t(p.mask_heads == 1 ? 0 : h) * p.nb + i;
+  int32_t start;
+  bool bad;
+  const int n = csr_row(p, csr, start, bad);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(bar_kv_full(s), 1); mbar_init(bar_kv_empty(s), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(bar_s_full(b), 1); mbar_init(bar_s_free(b), 4); }
+    mbar_init(bar_p_full, 4);
+    mbar_init(bar_o_done, 1);
+    mbar_init(bar_final, 1);
+    *abort_flag = 0;
+    *never = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) { tmem_alloc(smem_u32(tmem_slot), kTmemCols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
+      const int32_t q_row = int32_t(plane * p.n_pad + int64_t(i) * BN);
+      mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+      for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * BM * 128, &tm_q, c * 64, q_row, bar_q);
+      int issued = 0;
+      for (int t = 0; t < n; ++t) {
+        const int s = t % C::STAGES;
+        if (t >= C::STAGES && !mbar_wait(bar_kv_empty(s), ((t / C::STAGES) - 1) & 1, abort_flag)) {
+          *abort_flag = 1; report_fault(p.err, 5, 1); break;
+        }
+        const int32_t j = __ldg(p.col_idx + start + t);
+        const int32_t kv_row = int32_t(plane * p.n_pad + int64_t(j) * BN);
+        mbar_arrive_expect_tx(bar_kv_full(s), 2 * C::KV_BYTES);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_2d(sK + s * C::KV_BYTES + c * BN * 128, &tm_k, c * 64, kv_row, bar_kv_full(s));
+          tma_load_2d(sV + s * C::KV_BYTES + c * BN * 128, &tm_v, c * 64, kv_row, bar_kv_full(s));
+        }
+        issued = t + 1;
+      }
+      // After an abort, let the loads already issued land before the CTA exits.
+      if (*abort_flag) {
+        mbar_wait(bar_q, 0, never);
+        for (int t = (issued > C::STAGES ? issued - C::STAGES : 0); t < issued; ++t)
+          mbar_wait(bar_kv_full(t % C::STAGES), (t / C::STAGES) & 1, never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n > 0) {
+      bool ok = mbar_wait(bar_q, 0, abort_flag);
+      bool any_mma = false;
+      auto issue_pv = [&](int t) -> bool {
+        if (!mbar_wait(bar_p_full, t & 1, abort_flag)) return false;
+        tc_fence_after();
+        const int s = t % C::STAGES;
+        const uint32_t v_base = sV + s * C::KV_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t a = smem_desc_sw128(sP + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
+          const uint64_t b = smem_desc_sw128(v_base + kk * 16 * 128, BN * 128, 1024);
+          umma_f16_ss(tmem + C::TM_O, a, b, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar_kv_empty(s));
+        umma_commit(bar_o_done);
+        return true;
+      };
+      for (int t = 0; ok && t < n; ++t) {
+        const int s = t % C::STAGES, b = t & 1;
+        ok = mbar_wait(bar_kv_full(s), (t / C::STAGES) & 1, abort_flag);
+        if (ok && t >= 2) ok = mbar_wait(bar_s_free(b), ((t >> 1) - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t k_base = sK + s * C::KV_BYTES;
+        const uint32_t s_tm = tmem + (b ? C::TM_S1 : C::TM_S0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = smem_desc_sw128(sQ + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(k_base + (kk / 4) * BN * 128 + (kk % 4) * 32, 16, 1024);
+          umma_f16_ss(s_tm, a, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar_s_full(b));
+        any_mma = true;
+        if (t >= 1) ok = issue_pv(t - 1);
+      }
+      if (ok) ok = issue_pv(n - 1);
+      if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 2); }
+      if (any_mma) {
+        // Drain: every MMA issued by this thread completes before TMEM is released.
+        umma_commit(bar_final);
+        mbar_wait(bar_final, 0, never);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int sub = warp & 3;                     // TMEM lane quarter this warp may access
+    const int row = sub * 32 + lane;              // row of the 128-row tile
+    const uint32_t lane_off = uint32_t(sub * 32) << 16;
+    float m_ref = -INFINITY;                      // running max in log2 units (lazy)
+    float l = 0.f;
+    bool ok = true;
+    if (bad && threadIdx.x == kSoftmaxWarp0 * 32) report_fault(p.err, 1, int(csr & 0x7fffffff));
+
+    for (int t = 0; t < n; ++t) {
+      const int b = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), (t >> 1) & 1, abort_flag))) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[BN];
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c)
+        tmem_ld32(tmem + lane_off + (b ? C::TM_S1 : C::TM_S0) + c * 32,
+                  *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_s_free(b));
+
+      const int32_t j = __ldg(p.col_idx + start + t);
+      const int64_t valid = p.n_valid - int64_t(j) * BN;   // keys of this block that are real
+      float x[BN];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        x[c] = (c < valid) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+        mx = fmaxf(mx, x[c]);
+      }
+      const float m_old = m_ref;
+      if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
+      const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      float rs = 0.f;
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        const float p0 = ex2_approx(x[c] - m_use), p1 = ex2_approx(x[c + 1] - m_use);
+        rs += p0 + p1;
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      l = l * alpha + rs;
+
+      // P and O belong to the previous P*V product until it has completed.
+      if (t >= 1) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (t - 1) & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t ov[32];
+            tmem_ld32(tmem + lane_off + C::TM_O + c * 32, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(tmem + lane_off + C::TM_O + c * 32, ov);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P row -> shared memory, 128-byte swizzled K-major tile (64 keys per 128-byte slice).
+#pragma unroll
+      for (int c8 = 0; c8 < BN / 8; ++c8) {
+        const int box = c8 >> 3, chunk = c8 & 7;
+        const uint32_t addr = sP + box * (BM * 128) + row * 128 + ((chunk ^ (row & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[c8 * 4]),
+                     "r"(pk[c8 * 4 + 1]), "r"(pk[c8 * 4 + 2]), "r"(pk[c8 * 4 + 3])
+                     : "memory");
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok && n > 0) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (n - 1) & 1, abort_flag))) ok = false;
+      else tc_fence_after();
+    }
+    if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 3); }
+    const int64_t grow = int64_t(i) * BN + row;           // row within the plane
+    const bool store = row < BN && grow < p.n_pad;
+    const bool have = ok && n > 0 && l > 0.f;
+    const float inv_l = have ? 1.f / l : 0.f;
+    __nv_bfloat16* orow = p.o + (plane * p.n_pad + grow) * D;
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      if (ok && n > 0) {
+        tmem_ld32(tmem + lane_off + C::TM_O + c * 32, ov);
+        tmem_wait_ld();
+      }
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        w[e] = have ? pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l) : 0u;
+      if (store) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+      }
+    }
+    if (store) p.lse[plane * p.n_pad + grow] = have ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2D view [rows, d] of a bf16 [B, H, n_pad, d] tensor; box = 64 elements x box_rows.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+  const cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BN>
+cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why) {
+  using C = Cfg<D, BN>;
+  const int64_t rows = int64_t(a.B) * a.H * a.n_pad;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, a.q, rows, D, BM) || !make_map(&tk, a.k, rows, D, BN) ||
+      !make_map(&tv, a.v, rows, D, BN)) {
+    *why = "cuTensorMapEncodeTiled failed or is unavailable";
+    return cudaErrorInvalidValue;
+  }
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_BYTES);
+    if (e != cudaSuccess) { *why = "cudaFuncSetAttribute(max dynamic smem) failed"; return e; }
+    attr_set[dev] = true;
+  }
+  AttnParams p;
+  p.H = a.H;
+  p.nb = int(a.n_pad / a.block_size);
+  p.mask_heads = a.mask_heads;
+  p.n_pad = a.n_pad;
+  p.n_valid = a.n_valid;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.row_ptr = a.row_ptr;
+  p.col_idx = a.col_idx;
+  p.col_len = a.col_len;
+  p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.lse = a.lse;
+  p.err = a.err;
+  const int64_t items = rows / a.block_size;
+  if (items == 0) return cudaSuccess;
+  bsa_fwd_kernel<D, BN><<<dim3(unsigned(items)), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why) {
+  if (a.d == 128 && a.block_size == 128) return launch_cfg<128, 128>(a, stream, why);
+  if (a.d == 128 && a.block_size == 64) return launch_cfg<128, 64>(a, stream, why);
+  if (a.d == 64 && a.block_size == 128) return launch_cfg<64, 128>(a, stream, why);
+  if (a.d == 64 && a.block_size == 64) return launch_cfg<64, 64>(a, stream, why);
+  *why = "unsupported (d, block_size)";
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace lva

@@ -1,0 +1,109 @@
+"""One attention layer's hot path over the C ABI: tile reorder -> CSR -> attention -> inverse.
+
+``VideoBlockSparseAttention`` owns the device buffers of a fixed problem shape (allocated
+once through torch, which is used only for device memory and streams) and runs, per call:
+
+1. ``lva_reorder_tokens`` on Q, K and V (raster [B, H, N, d] -> tile order [B, H, n_pad, d]);
+2. ``lva_build_block_mask`` for the current denoising step (window + rotating anchors
+   change with the step; static, two-stage and all-ones masks are built once);
+3. ``lva_block_sparse_attn`` -> O (tile order) and LSE;
+4. ``lva_reorder_tokens`` inverse on O (tile order -> raster [B, H, N, d]).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _binding as lb
+
+
+def mask_params_for(spec: dict, n_pad: int, n_valid: int, block_size: int, mask_heads: int = 1,
+                    step: int = 0) -> lb.MaskParams:
+    """``MaskParams`` for a mask specification dict (kind, unit, radius, anchors, group)."""
+    kind = spec["kind"]
+    if kind == "window_anchor":
+        return lb.MaskParams(lb.LVA_MASK_WINDOW_ANCHOR, n_pad, n_valid, block_size, 1,
+                             spec["unit"], spec["radius"], spec["anchors"], step)
+    if kind == "two_stage":
+        return lb.MaskParams(lb.LVA_MASK_TWO_STAGE, n_pad, n_valid, block_size, 1, group_blocks=spec["group"])
+    if kind == "all":
+        return lb.MaskParams(lb.LVA_MASK_ALL, n_pad, n_valid, block_size, 1)
+    if kind == "static":
+        return lb.MaskParams(lb.LVA_MASK_STATIC, n_pad, n_valid, block_size, mask_heads)
+    raise ValueError(f"unknown mask kind {kind!r}")
+
+
+class VideoBlockSparseAttention:
+    """Block-sparse self-attention over a T x Hg x Wg latent video grid.
+
+    ``mask`` is a specification dict; for ``kind == "static"`` pass the dense per-head block
+    mask (uint8 [H_m, nb, nb], any device) as ``static_mask``.
+    """
+
+    def __init__(self, B, H, d, grid, tile, block_size, mask: dict, static_mask=None,
+                 scale=None, device="cuda"):
+        self.B, self.H, self.d = B, H, d
+        self.grid, self.tile, self.block_size = tuple(grid), tuple(tile), block_size
+        self.n_valid = grid[0] * grid[1] * grid[2]
+        self.n_pad = (self.n_valid + block_size - 1) // block_size * block_size
+        self.nb = self.n_pad // block_size
+        self.mask = dict(mask)
+        self.scale = float(scale) if scale is not None else float(torch.tensor(d ** -0.5, dtype=torch.float32))
+        self.device = torch.device(device)
+        self.mask_heads = 1
+        self.dense_mask = None
+        if mask["kind"] == "static":
+            if static_mask is None:
+                raise ValueError("static mask kind needs static_mask")
+            sm = torch.as_tensor(static_mask, dtype=torch.uint8)
+            self.mask_heads = sm.shape[0]
+            self.dense_mask = sm.to(self.device).contiguous()
+        self.params = mask_params_for(self.mask, self.n_pad, self.n_valid, block_size, self.mask_heads)
+        cap = lb.lva_block_mask_max_nnz(self.params)
+        if cap <= 0:
+            raise ValueError(f"invalid mask parameters {self.params}")
+        kw = dict(device=self.device)
+        shape = (B, H, self.n_pad, d)
+        self.q_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
+        self.k_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
+        self.v_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
+        self.o_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
+        self.lse = torch.empty((B, H, self.n_pad), dtype=torch.float32, **kw)
+        self.o = torch.empty((B, H, self.n_valid, d), dtype=torch.bfloat16, **kw)
+        self.row_ptr = torch.empty(self.mask_heads * self.nb + 1, dtype=torch.int32, **kw)
+        self.col_idx = torch.empty(cap, dtype=torch.int32, **kw)
+        self.nnz = torch.empty(1, dtype=torch.int32, **kw)
+        self._built_step = None
+
+    def build_mask(self, step: int = 0):
+        """(Re)build the CSR; parametric window masks depend on the denoising step."""
+        steps_matter = self.mask["kind"] == "window_anchor" and self.mask.get("anchors", 0) > 0
+        key = step if steps_matter else 0
+        if self._built_step == key:
+            return
+        self.params.step = key
+        lb.lva_build_block_mask(self.params, self.dense_mask, self.row_ptr, self.col_idx, self.nnz)
+        self._built_step = key
+
+    def reorder_in(self, q, k, v):
+        P = self.B * self.H
+        for src, dst in ((q, self.q_t), (k, self.k_t), (v, self.v_t)):
+            lb.lva_reorder_tokens(src.view(P, self.n_valid, self.d), dst.view(P, self.n_pad, self.d),
+                                  self.grid, self.tile, self.n_pad, inverse=False)
+
+    def attend(self):
+        lb.lva_block_sparse_attn(self.q_t, self.k_t, self.v_t, self.o_t, self.lse, self.n_valid,
+                                 self.block_size, self.row_ptr, self.col_idx, self.mask_heads, self.scale)
+
+    def reorder_out(self):
+        P = self.B * self.H
+        lb.lva_reorder_tokens(self.o_t.view(P, self.n_pad, self.d), self.o.view(P, self.n_valid, self.d),
+                              self.grid, self.tile, self.n_pad, inverse=True)
+
+    def __call__(self, q, k, v, step: int = 0):
+        """Raster-order bf16 Q, K, V [B, H, N, d] on this device -> raster O (the internal
+        buffer ``self.o``) and tile-order LSE ``self.lse``."""
+        self.reorder_in(q, k, v)
+        self.build_mask(step)
+        self.attend()
+        self.reorder_out()
+        return self.o, self.lse

@@ -1,0 +1,183 @@
+/*
+ * lva.h -- block-sparse softmax attention for video diffusion transformers on B200 (sm_100a).
+ *
+ * C ABI.  Every pointer argument named as "device" is a device address of the current CUDA
+ * device; every call is asynchronous on the given stream and returns after argument checks
+ * and kernel launch.  The library allocates no memory: the caller owns every buffer.
+ *
+ * Errors: a call returns LVA_OK or a status code.  Argument errors are found on the host
+ * before anything is launched (nothing is written in that case).  A failed launch returns
+ * LVA_ERR_CUDA.  Faults found by the kernels themselves (a CSR entry out of range, a wait
+ * that ran past its time limit) are recorded in a per-device error word that
+ * lva_device_error() reads; the kernels then skip the bad work instead of touching memory
+ * outside the buffers.  lva_last_error_message() gives a one-line explanation of the
+ * last failure on the calling thread.
+ *
+ * Layouts:
+ *   tokens   -- a plane (one batch element and head) is n rows of row_elems elements;
+ *               planes are contiguous: element (p, r, e) sits at ((p*n + r)*row_elems + e).
+ *   Q, K, V, O -- bf16 [B, H, n_pad, d], row-major, rows in tile order (see
+ *               lva_reorder_tokens), rows n_valid..n_pad-1 are padding.
+ *   LSE      -- fp32 [B, H, n_pad].
+ *   CSR      -- row r = h_m*nb + i lists the key blocks j that query block i attends under
+ *               mask head h_m: col_idx[row_ptr[r] .. row_ptr[r+1]-1], ascending, unique.
+ */
+#ifndef LVA_H
+#define LVA_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LVA_VERSION 1
+
+typedef enum {
+  LVA_OK = 0,
+  LVA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, inconsistent sizes, bad CSR */
+  LVA_ERR_UNSUPPORTED = 2,   /* a size or mode this build has no kernel for */
+  LVA_ERR_CAPACITY = 3,      /* an output buffer is too small */
+  LVA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+  LVA_ERR_TIMEOUT = 5        /* a kernel wait ran past its limit (device error word) */
+} lva_status;
+
+/* Human-readable name of a status code (static string). */
+const char* lva_status_string(lva_status status);
+
+/* One-line description of the last failure on the calling thread ("" if none). */
+const char* lva_last_error_message(void);
+
+/* LVA_VERSION of the loaded library. */
+int lva_version(void);
+
+/*
+ * lva_reorder_tokens -- spatiotemporal-tile token order and its inverse.
+ *
+ * Defines the token order in which blocks of the attention matrix are spatiotemporal
+ * neighbourhoods, the granularity at which the LVSA page ("LVSA: Training-Free Sparse
+ * Attention for Long Video Diffusion", technical summary section 2, "Meccanismo Core")
+ * restricts a query frame's attended set, and at which the CalibAtt page ("Accelerating
+ * Text-to-Video Generation with Calibrated Sparse Attention", section 2, step A.1) cuts
+ * the matrix into 128x128 blocks.  The order: tiles of tile_t x tile_h x tile_w latent
+ * tokens, enumerated in raster order of tile coordinates; tokens in raster order inside a
+ * tile; edge tiles are partial (no per-tile padding).
+ *
+ * With N = T*H*W and perm[k] the raster index t*H*W + h*W + w of the k-th token in tile
+ * order:
+ *   inverse == 0:  src [planes, N, row] (raster) -> dst [planes, n_pad, row] (tile order):
+ *                  dst[p][k] = src[p][perm[k]] for k < N; rows N..n_pad-1 are zeroed.
+ *   inverse != 0:  src [planes, n_pad, row] (tile order) -> dst [planes, N, row] (raster):
+ *                  dst[p][perm[k]] = src[p][k] for k < N; src rows >= N are ignored.
+ * Rows are copied bit for bit.  row = row_elems elements of elem_bytes (2 or 4) bytes.
+ *
+ * src, dst: device, must not overlap, aligned to elem_bytes.  n_pad >= N.
+ * planes * n_pad * row_elems * elem_bytes must fit in int64.
+ * Errors: LVA_ERR_INVALID_ARG for null pointers, non-positive sizes, n_pad < N, bad
+ * elem_bytes or misalignment.  planes == 0 is a no-op.
+ */
+lva_status lva_reorder_tokens(const void* src, void* dst, int64_t planes,
+                              int T, int H, int W, int tile_t, int tile_h, int tile_w,
+                              int64_t n_pad, int64_t row_elems, int elem_bytes, int inverse,
+                              cudaStream_t stream);
+
+/* Block-mask kinds for lva_build_block_mask. */
+typedef enum {
+  LVA_MASK_WINDOW_ANCHOR = 0,  /* local window + rotating global anchors (LVSA)      */
+  LVA_MASK_STATIC = 1,         /* a given dense per-head block mask (CalibAtt-style) */
+  LVA_MASK_ALL = 2,            /* every block: dense attention                       */
+  LVA_MASK_TWO_STAGE = 3       /* local window groups + one strided block (SQuad-style) */
+} lva_mask_kind;
+
+typedef struct {
+  int kind;                    /* lva_mask_kind */
+  int mask_heads;              /* H_m: rows of masks built; 1 unless kind is STATIC */
+  int block_size;              /* Bs: 64 or 128 tokens */
+  int64_t n_pad;               /* padded sequence length, a multiple of block_size */
+  int64_t n_valid;             /* real tokens, 1 <= n_valid <= n_pad */
+  int64_t window_unit_tokens;  /* WINDOW_ANCHOR: U, tokens per window unit (H*W = frames) */
+  int window_radius;           /* WINDOW_ANCHOR: r >= 0, in units */
+  int num_anchors;             /* WINDOW_ANCHOR: G >= 0 anchor key blocks */
+  int step;                    /* WINDOW_ANCHOR: denoising step s >= 0 */
+  int group_blocks;            /* TWO_STAGE: g >= 1 blocks per local window group */
+} lva_mask_params;
+
+/* Upper bound on the CSR entries of a mask: mask_heads * nb * nb (0 on bad params). */
+int64_t lva_block_mask_max_nnz(const lva_mask_params* params);
+
+/*
+ * lva_build_block_mask -- per-query-block CSR lists of the key blocks to compute.
+ *
+ * The CSR is the skip list of the CalibAtt page ("Accelerating Text-to-Video Generation
+ * with Calibrated Sparse Attention", section 2 B, "Fase di Inferenza": precomputed lists of
+ * blocks per (timestep, layer, head), deterministic, no decision at inference time), built
+ * on the GPU from one of these masks, with nb = n_pad / block_size:
+ *
+ *   WINDOW_ANCHOR (LVSA page, technical summary section 2, "Meccanismo Core":
+ *     A(t) = G union W(t); the global set G_s moves by s mod T_per at step s).
+ *     Block i covers window units lo(i) = floor(i*Bs/U) .. hi(i) = floor((min((i+1)*Bs,
+ *     n_valid) - 1)/U); a block of padding only takes the unit of the last real token.
+ *     Anchors G_s = { (floor(a*nb/G) + s) mod nb : a < G }.
+ *     M[i][j] = (lo(j) <= hi(i) + r  and  hi(j) >= lo(i) - r)  or  j in G_s.
+ *   STATIC: M[h][i][j] = dense_mask[(h*nb + i)*nb + j] != 0, used as given.
+ *   ALL:    M[i][j] = 1.
+ *   TWO_STAGE (SQuad page, "SQuad: Sub-Quadratic Attention Distillation for Efficient
+ *     Video Generation", technical summary section 1: local pass in windows of w tokens,
+ *     global pass across windows at the same relative position):
+ *     M[i][j] = (floor(j/g) == floor(i/g))  or  j == (i + g) mod nb.
+ *
+ * Outputs (device): row_ptr [mask_heads*nb + 1] (row_ptr[0] = 0), col_idx [col_capacity],
+ * *nnz_out = row_ptr[mask_heads*nb].  Columns of a row are ascending and unique.
+ * dense_mask (device) is read only for STATIC ([mask_heads, nb, nb] uint8) and may be NULL
+ * otherwise.
+ * Errors: LVA_ERR_INVALID_ARG for bad parameters or pointers; LVA_ERR_CAPACITY when
+ * col_capacity < lva_block_mask_max_nnz(params) (nothing is launched).
+ */
+lva_status lva_build_block_mask(const lva_mask_params* params, const uint8_t* dense_mask,
+                                int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                int32_t* nnz_out, cudaStream_t stream);
+
+/*
+ * lva_block_sparse_attn -- softmax attention computed only on listed block pairs.
+ *
+ * The block-sparse attention of the LVSA page (technical summary section 2: attention
+ * restricted to A(t) through a block-sparse mechanism) and of the CalibAtt page (section
+ * 2 B: non-repetitive heads attend only the selected blocks of the skip list).  For batch
+ * b, head h and query row r in block i = r / Bs, with h_m = (mask_heads == 1 ? 0 : h):
+ *   J   = { c : c < n_valid and c / Bs is listed in CSR row h_m*nb + i }
+ *   s_c = scale * <q_r, k_c>;  m = max_c s_c;  l = sum_c exp(s_c - m)
+ *   O_r = sum_c exp(s_c - m) v_c / l   (bf16, round to nearest even)
+ *   LSE_r = m + ln(l)                  (fp32, natural log, scale included)
+ * An empty J gives O_r = 0 and LSE_r = -inf.  Padded query rows are computed like the rest.
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation; probabilities are rounded
+ * to bf16 before the P*V product; softmax statistics are fp32.
+ *
+ * q, k, v, o: device bf16 [B, H, n_pad, d], 16-byte aligned.  lse: device fp32 [B, H, n_pad].
+ * row_ptr: device [mask_heads*nb + 1]; col_idx: device, col_len entries (the kernel never
+ * reads past col_len; CSR entries out of range are skipped and reported through
+ * lva_device_error as LVA_ERR_INVALID_ARG).
+ * Supported: d in {64, 128}, block_size in {64, 128}, mask_heads in {1, H},
+ * B*H*n_pad < 2^31.
+ */
+lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 int B, int H, int64_t n_pad, int64_t n_valid, int d,
+                                 int block_size, const int32_t* row_ptr, const int32_t* col_idx,
+                                 int64_t col_len, int mask_heads, float scale,
+                                 cudaStream_t stream);
+
+/*
+ * lva_device_error -- read and clear the current device's kernel error word.
+ *
+ * Synchronises `stream`, then stores in *status the first kernel-side fault recorded since
+ * the last call (LVA_OK if none): LVA_ERR_INVALID_ARG for CSR entries out of range,
+ * LVA_ERR_TIMEOUT for a pipeline wait that ran past its limit.  *detail (may be NULL)
+ * receives a kernel-specific code locating the fault.
+ */
+lva_status lva_device_error(cudaStream_t stream, lva_status* status, int* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LVA_H */

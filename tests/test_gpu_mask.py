@@ -1,0 +1,112 @@
+"""GPU block-mask -> CSR vs the oracle: bit-exact row_ptr, col_idx and nnz."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle.mask import all_mask, dense_to_csr, two_stage_mask, window_anchor_mask
+from synthetic import WORKLOADS, mask_variants, static_calibrated_mask
+from tests.gpu_helpers import require_gpu
+
+pytestmark = pytest.mark.gpu
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _build(params, dense=None):
+    import block_sparse_attention_lva_b200 as lva
+    dev = require_gpu()
+    nb = params.n_pad // params.block_size
+    cap = lva.lva_block_mask_max_nnz(params)
+    row_ptr = torch.full((params.mask_heads * nb + 1,), -5, dtype=torch.int32, device=dev)
+    col_idx = torch.full((cap,), -5, dtype=torch.int32, device=dev)
+    nnz = torch.zeros(1, dtype=torch.int32, device=dev)
+    dm = torch.from_numpy(np.ascontiguousarray(dense, dtype=np.uint8)).to(dev) if dense is not None else None
+    lva.lva_build_block_mask(params, dm, row_ptr, col_idx, nnz)
+    torch.cuda.synchronize()
+    rp = row_ptr.cpu().numpy()
+    n = int(nnz.item())
+    assert n == rp[-1]
+    return rp, col_idx.cpu().numpy()[:n]
+
+
+def _check(params, ref_masks, dense=None):
+    rp, ci = _build(params, dense)
+    rp_ref, ci_ref = dense_to_csr(ref_masks)
+    assert np.array_equal(rp, rp_ref)
+    assert np.array_equal(ci, ci_ref)
+
+
+def test_tiny_golden():
+    import block_sparse_attention_lva_b200 as lva
+    g = json.load(open(os.path.join(GOLDEN, "mask_tiny.json")))
+    p = lva.MaskParams(lva.LVA_MASK_WINDOW_ANCHOR, g["n_pad"], g["n_valid"], g["block_size"], 1,
+                       g["unit_tokens"], g["radius"], g["num_anchors"], g["step"])
+    rp, ci = _build(p)
+    assert rp.tolist() == g["row_ptr"] and ci.tolist() == g["col_idx"]
+
+
+def test_small_every_step():
+    import block_sparse_attention_lva_b200 as lva
+    w = WORKLOADS["small"]
+    spec = mask_variants(w)[0]
+    for s in spec["steps"]:
+        p = lva.MaskParams(lva.LVA_MASK_WINDOW_ANCHOR, w.n_pad, w.n_valid, w.block_size, 1,
+                           spec["unit"], spec["radius"], spec["anchors"], s)
+        _check(p, window_anchor_mask(w.n_pad, w.n_valid, w.block_size, spec["unit"], spec["radius"],
+                                     spec["anchors"], s))
+
+
+def test_static_and_all():
+    import block_sparse_attention_lva_b200 as lva
+    w = WORKLOADS["static"]
+    dense = static_calibrated_mask(w)
+    p = lva.MaskParams(lva.LVA_MASK_STATIC, w.n_pad, w.n_valid, w.block_size, w.H)
+    _check(p, dense.astype(bool), dense)
+    _check(lva.MaskParams(lva.LVA_MASK_ALL, w.n_pad, w.n_valid, w.block_size), all_mask(w.nb))
+
+
+@pytest.mark.parametrize("name", ["large", "long"])
+def test_sweeps(name):
+    import block_sparse_attention_lva_b200 as lva
+    w = WORKLOADS[name]
+    for spec in mask_variants(w):
+        if spec["kind"] == "window_anchor":
+            p = lva.MaskParams(lva.LVA_MASK_WINDOW_ANCHOR, w.n_pad, w.n_valid, w.block_size, 1,
+                               spec["unit"], spec["radius"], spec["anchors"], 0)
+            ref = window_anchor_mask(w.n_pad, w.n_valid, w.block_size, spec["unit"], spec["radius"],
+                                     spec["anchors"], 0)
+        elif spec["kind"] == "two_stage":
+            p = lva.MaskParams(lva.LVA_MASK_TWO_STAGE, w.n_pad, w.n_valid, w.block_size, 1,
+                               group_blocks=spec["group"])
+            ref = two_stage_mask(w.nb, spec["group"])
+        else:
+            p = lva.MaskParams(lva.LVA_MASK_ALL, w.n_pad, w.n_valid, w.block_size)
+            ref = all_mask(w.nb)
+        _check(p, ref)
+
+
+def test_edge_cases():
+    import block_sparse_attention_lva_b200 as lva
+    rng = np.random.default_rng(9)
+    # Static masks whose rows are not 16-byte multiples (byte path), with empty rows.
+    for hm, nb in [(3, 37), (2, 1), (1, 600)]:
+        dense = (rng.random((hm, nb, nb)) < 0.2).astype(np.uint8)
+        dense[0, 0] = 0
+        p = lva.MaskParams(lva.LVA_MASK_STATIC, nb * 64, nb * 64 - 5, 64, hm)
+        _check(p, dense.astype(bool), dense)
+    # Static, vector path, a row entirely empty and one entirely full.
+    dense = (rng.random((2, 64, 64)) < 0.5).astype(np.uint8)
+    dense[1, 3] = 0
+    dense[1, 4] = 1
+    _check(lva.MaskParams(lva.LVA_MASK_STATIC, 64 * 128, 64 * 128, 128, 2), dense.astype(bool), dense)
+    # Window masks with trailing padding-only blocks, radius 0, anchors beyond the window,
+    # large step, many anchors.
+    for (n_pad, n_valid, bs, U, r, G, s) in [(1024, 700, 64, 100, 0, 3, 123), (4096, 4096, 128, 128, 0, 32, 5),
+                                            (8192, 5000, 128, 1560, 2, 1, 0), (640, 64, 64, 64, 1, 10, 7)]:
+        p = lva.MaskParams(lva.LVA_MASK_WINDOW_ANCHOR, n_pad, n_valid, bs, 1, U, r, G, s)
+        _check(p, window_anchor_mask(n_pad, n_valid, bs, U, r, G, s))
+    for nb, g in [(10, 3), (7, 7), (5, 1), (9, 20)]:
+        p = lva.MaskParams(lva.LVA_MASK_TWO_STAGE, nb * 128, nb * 128, 128, 1, group_blocks=g)
+        _check(p, two_stage_mask(nb, g))
