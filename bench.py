@@ -134,6 +134,17 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def reduce_over_ranks(times, work, device, distributed: bool):
+    """Max over ranks of each time, sum over ranks of the work (the only cross-rank traffic)."""
+    t = torch.tensor(list(times), dtype=torch.float64, device=device)
+    wk = torch.tensor([float(work)], dtype=torch.float64, device=device)
+    if distributed:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(wk, op=dist.ReduceOp.SUM)
+    return t.tolist(), wk.item()
+
+
 def _flops_per_nnz(w: Workload) -> float:
     return 4.0 * w.block_size * w.block_size * w.d
 
@@ -241,13 +252,8 @@ def run_lva(args):
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
 
     # ---------------- reduce over ranks (max time, summed work)
-    times = torch.tensor([ms_total, ms_e2e, float(np.mean(attn_ms))], dtype=torch.float64, device=dev)
-    work = torch.tensor([flops], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(times, op=dist.ReduceOp.MAX)
-        dist.all_reduce(work, op=dist.ReduceOp.SUM)
-    ms_total, ms_e2e, attn_ms_mean = times.tolist()
-    flops_all = work.item()
+    (ms_total, ms_e2e, attn_ms_mean), flops_all = reduce_over_ranks(
+        [ms_total, ms_e2e, float(np.mean(attn_ms))], flops, dev, ws > 1)
 
     if rank == 0:
         burst, sustained, hbm, peak_kind = _peaks()
