@@ -7,14 +7,16 @@
 // technical summary section 2) -- with an online softmax, so the cost is proportional to
 // the number of listed blocks.
 //
-// Warp roles (192 threads):
-//   warp 0      TMA producer: Q tile once, then K_j / V_j tiles into a STAGES-deep ring;
+// Warp roles (352 threads):
+//   warp 0      TMA producer: Q tile once, then K_j tiles into a 3-slot ring;
+//   warp 10     TMA producer: V_j tiles into a 2-slot ring;
 //   warp 1      MMA issuer (one thread): S = Q K_j^T into TMEM (two S buffers), and
 //               O += P V_j into a TMEM accumulator; owns the TMEM allocation;
-//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane = row): read S
-//               from TMEM, update running max / sum, write P (bf16) to shared memory in
-//               the tensor-core operand layout, rescale O in TMEM when the max moves by
-//               more than 2^8, and finally normalise O and write O and LSE.
+//   warps 2..9  softmax + epilogue, one (query row, column half) per thread (TMEM lane =
+//               row): read S from TMEM, update the running max (shared by the two halves
+//               of a row) and sum, write P (bf16) to shared memory in the tensor-core
+//               operand layout, rescale O in TMEM when the max moves by more than 2^8, and
+//               finally normalise O and write O and LSE.
 //
 // Shared-memory operands use the 128-byte swizzle that TMA writes: a 64-element (128 B)
 // slice of each row, eight rows per 1024-byte atom.  Q, K and P are K-major; V is read
@@ -30,8 +32,10 @@ namespace lva {
 namespace {
 
 constexpr int BM = 128;            // query rows per MMA tile (TMEM lanes)
-constexpr int kThreads = 192;
 constexpr int kSoftmaxWarp0 = 2;
+constexpr int kSoftmaxWarps = 8;   // two warps per TMEM lane quarter: one per column half
+constexpr int kVWarp = kSoftmaxWarp0 + kSoftmaxWarps;   // V producer, after the softmax warps
+constexpr int kThreads = 32 * (kVWarp + 1);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when max grows > 2^8
 constexpr uint32_t kTmemCols = 512;
 
@@ -49,22 +53,29 @@ struct AttnParams {
 
 template <int D, int BN>
 struct Cfg {
-  static constexpr int STAGES = 2;
+  // K and V live in separate rings: a K slot is free once Q*K^T has read it, a V slot only
+  // after P*V, so K loads run further ahead than V loads.
+  static constexpr int KST = 3, VST = 2;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_P = OFF_V + VST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], s_free[2], p_full, o_done, final
-  static constexpr int NUM_BARS = 1 + 2 * STAGES + 2 + 2 + 1 + 1 + 1;
+  // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2],
+  // s_free[2], p_full, o_done, final, pair[4 lane quarters][2 slots]
+  static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST, B_VE = B_VF + VST,
+                       B_SF = B_VE + VST, B_SE = B_SF + 2, B_P = B_SE + 2, B_O = B_P + 1,
+                       B_FIN = B_O + 1, B_PAIR = B_FIN + 1, NUM_BARS = B_PAIR + 8;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  // + slack for 1024-byte alignment; at least 120 KB so that one CTA (and one 512-column
-  // TMEM allocation) is resident per SM.
-  static constexpr int SMEM_RAW = OFF_MISC + 16 + 1024;
+  // row-max / row-sum exchange between the two column halves: [2 slots][2 halves][BM] floats
+  static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
+  // At least 120 KB so that one CTA (and one 512-column TMEM allocation) is resident per SM.
+  static constexpr int SMEM_RAW = OFF_RED + 2 * 2 * BM * 4;
   static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
@@ -95,20 +106,27 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = Cfg<D, BN>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 128-byte-swizzled TMA tiles need 1024-byte aligned shared memory.
+  extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t s_base = smem_u32(smem);
+  if (s_base & 1023u) {                           // never expected; checked rather than assumed
+    if (threadIdx.x == 0) report_fault(p.err, 4, 1023);
+    return;
+  }
   const uint32_t sQ = s_base + C::OFF_Q, sK = s_base + C::OFF_K, sV = s_base + C::OFF_V,
                  sP = s_base + C::OFF_P;
   const uint32_t bar0 = s_base + C::OFF_BAR;
-  const uint32_t bar_q = bar0;
-  auto bar_kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
-  auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + C::STAGES + s); };
-  auto bar_s_full = [&](int b) { return bar0 + 8u * (1 + 2 * C::STAGES + b); };
-  auto bar_s_free = [&](int b) { return bar0 + 8u * (3 + 2 * C::STAGES + b); };
-  const uint32_t bar_p_full = bar0 + 8u * (5 + 2 * C::STAGES);
-  const uint32_t bar_o_done = bar0 + 8u * (6 + 2 * C::STAGES);
-  const uint32_t bar_final = bar0 + 8u * (7 + 2 * C::STAGES);
+  const uint32_t bar_q = bar0 + 8u * C::B_Q;
+  auto bar_k_full = [&](int s) { return bar0 + 8u * (C::B_KF + s); };
+  auto bar_k_empty = [&](int s) { return bar0 + 8u * (C::B_KE + s); };
+  auto bar_v_full = [&](int s) { return bar0 + 8u * (C::B_VF + s); };
+  auto bar_v_empty = [&](int s) { return bar0 + 8u * (C::B_VE + s); };
+  auto bar_s_full = [&](int b) { return bar0 + 8u * (C::B_SF + b); };
+  auto bar_s_free = [&](int b) { return bar0 + 8u * (C::B_SE + b); };
+  const uint32_t bar_p_full = bar0 + 8u * C::B_P;
+  const uint32_t bar_o_done = bar0 + 8u * C::B_O;
+  const uint32_t bar_final = bar0 + 8u * C::B_FIN;
+  auto bar_pair = [&](int q, int slot) { return bar0 + 8u * (C::B_PAIR + 2 * q + slot); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   // Stays zero: the drain waits after an abort are bounded by time alone.
@@ -128,11 +146,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < C::STAGES; ++s) { mbar_init(bar_kv_full(s), 1); mbar_init(bar_kv_empty(s), 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(bar_s_full(b), 1); mbar_init(bar_s_free(b), 4); }
-    mbar_init(bar_p_full, 4);
+    for (int s = 0; s < C::KST; ++s) { mbar_init(bar_k_full(s), 1); mbar_init(bar_k_empty(s), 1); }
+    for (int s = 0; s < C::VST; ++s) { mbar_init(bar_v_full(s), 1); mbar_init(bar_v_empty(s), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(bar_s_full(b), 1); mbar_init(bar_s_free(b), kSoftmaxWarps); }
+    mbar_init(bar_p_full, kSoftmaxWarps);
     mbar_init(bar_o_done, 1);
     mbar_init(bar_final, 1);
+    for (int q = 0; q < 4; ++q) { mbar_init(bar_pair(q, 0), 2); mbar_init(bar_pair(q, 1), 2); }
     *abort_flag = 0;
     *never = 0;
     mbar_fence_init();
@@ -143,34 +163,42 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  // One TMA producer loop: tile t of `n` goes to slot t % ST of a ring whose slots are
+  // released by `empty` barriers; after an abort, waits for the loads already issued.
+  auto produce = [&](const void* tmap, uint32_t ring, int ST, uint32_t full0, uint32_t empty0, int code) {
+    int issued = 0;
+    for (int t = 0; t < n; ++t) {
+      const int s = t % ST;
+      if (t >= ST && !mbar_wait(empty0 + 8u * s, ((t / ST) - 1) & 1, abort_flag)) {
+        *abort_flag = 1; report_fault(p.err, 5, code); break;
+      }
+      const int32_t j = __ldg(p.col_idx + start + t);
+      const int32_t kv_row = int32_t(plane * p.n_pad + int64_t(j) * BN);
+      mbar_arrive_expect_tx(full0 + 8u * s, C::KV_BYTES);
+      for (int c = 0; c < D / 64; ++c)
+        tma_load_2d(ring + s * C::KV_BYTES + c * BN * 128, tmap, c * 64, kv_row, full0 + 8u * s);
+      issued = t + 1;
+    }
+    if (*abort_flag)
+      for (int t = (issued > ST ? issued - ST : 0); t < issued; ++t)
+        mbar_wait(full0 + 8u * (t % ST), (t / ST) & 1, never);
+  };
+
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer: Q, K
     if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k);
       const int32_t q_row = int32_t(plane * p.n_pad + int64_t(i) * BN);
       mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
       for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * BM * 128, &tm_q, c * 64, q_row, bar_q);
-      int issued = 0;
-      for (int t = 0; t < n; ++t) {
-        const int s = t % C::STAGES;
-        if (t >= C::STAGES && !mbar_wait(bar_kv_empty(s), ((t / C::STAGES) - 1) & 1, abort_flag)) {
-          *abort_flag = 1; report_fault(p.err, 5, 1); break;
-        }
-        const int32_t j = __ldg(p.col_idx + start + t);
-        const int32_t kv_row = int32_t(plane * p.n_pad + int64_t(j) * BN);
-        mbar_arrive_expect_tx(bar_kv_full(s), 2 * C::KV_BYTES);
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_2d(sK + s * C::KV_BYTES + c * BN * 128, &tm_k, c * 64, kv_row, bar_kv_full(s));
-          tma_load_2d(sV + s * C::KV_BYTES + c * BN * 128, &tm_v, c * 64, kv_row, bar_kv_full(s));
-        }
-        issued = t + 1;
-      }
-      // After an abort, let the loads already issued land before the CTA exits.
-      if (*abort_flag) {
-        mbar_wait(bar_q, 0, never);
-        for (int t = (issued > C::STAGES ? issued - C::STAGES : 0); t < issued; ++t)
-          mbar_wait(bar_kv_full(t % C::STAGES), (t / C::STAGES) & 1, never);
-      }
+      produce(&tm_k, sK, C::KST, bar_k_full(0), bar_k_empty(0), 1);
+      if (*abort_flag) mbar_wait(bar_q, 0, never);
+    }
+  } else if (warp == kVWarp) {
+    // ------------------------------------------------------------ TMA producer: V
+    if (lane == 0 && n > 0) {
+      tma_prefetch_desc(&tm_v);
+      produce(&tm_v, sV, C::VST, bar_v_full(0), bar_v_empty(0), 6);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -178,9 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       bool ok = mbar_wait(bar_q, 0, abort_flag);
       bool any_mma = false;
       auto issue_pv = [&](int t) -> bool {
+        const int s = t % C::VST;
         if (!mbar_wait(bar_p_full, t & 1, abort_flag)) return false;
+        if (!mbar_wait(bar_v_full(s), (t / C::VST) & 1, abort_flag)) return false;
         tc_fence_after();
-        const int s = t % C::STAGES;
         const uint32_t v_base = sV + s * C::KV_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
@@ -188,13 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           const uint64_t b = smem_desc_sw128(v_base + kk * 16 * 128, BN * 128, 1024);
           umma_f16_ss(tmem + C::TM_O, a, b, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(bar_kv_empty(s));
+        umma_commit(bar_v_empty(s));
         umma_commit(bar_o_done);
         return true;
       };
       for (int t = 0; ok && t < n; ++t) {
-        const int s = t % C::STAGES, b = t & 1;
-        ok = mbar_wait(bar_kv_full(s), (t / C::STAGES) & 1, abort_flag);
+        const int s = t % C::KST, b = t & 1;
+        ok = mbar_wait(bar_k_full(s), (t / C::KST) & 1, abort_flag);
         if (ok && t >= 2) ok = mbar_wait(bar_s_free(b), ((t >> 1) - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
@@ -207,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           umma_f16_ss(s_tm, a, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar_s_full(b));
+        umma_commit(bar_k_empty(s));
         any_mma = true;
         if (t >= 1) ok = issue_pv(t - 1);
       }
@@ -220,50 +250,107 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
+    // Thread = (query row, column half).  Warps w and w+4 share a TMEM lane quarter, so
+    // they own the same 32 rows; the first takes key/O columns [0, half), the second
+    // [half, 2*half).  They exchange the row max once per key block.
+    constexpr int HALF = BN / 2, DH = D / 2;
+    const int sw = warp - kSoftmaxWarp0;          // 0..7
+    const int hf = sw >> 2;                       // column half
     const int sub = warp & 3;                     // TMEM lane quarter this warp may access
     const int row = sub * 32 + lane;              // row of the 128-row tile
     const uint32_t lane_off = uint32_t(sub * 32) << 16;
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);   // [slot][half][row]
+    // Exchange of one value per row with the partner warp (other column half).  Exchange
+    // number `seq` uses slot seq & 1; the partner's read of a slot always precedes its
+    // arrival on the next exchange, so a slot is never overwritten before it is read.
+    auto pair_exchange = [&](int seq, float v, bool& good) -> float {
+      float* slot = red + (seq & 1) * 2 * BM;
+      slot[hf * BM + row] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pair(sub, seq & 1));
+      good = __all_sync(0xffffffffu, mbar_wait(bar_pair(sub, seq & 1), (seq >> 1) & 1, abort_flag));
+      return good ? slot[(1 - hf) * BM + row] : 0.f;
+    };
+    const float c = p.scale_log2;                 // scores -> log2 units
     float m_ref = -INFINITY;                      // running max in log2 units (lazy)
-    float l = 0.f;
+    float l = 0.f;                                // this half's share of the row sum
     bool ok = true;
     if (bad && threadIdx.x == kSoftmaxWarp0 * 32) report_fault(p.err, 1, int(csr & 0x7fffffff));
+    int32_t jn = n > 0 ? __ldg(p.col_idx + start) : 0;
 
     for (int t = 0; t < n; ++t) {
       const int b = t & 1;
+      const int32_t j = jn;
+      if (t + 1 < n) jn = __ldg(p.col_idx + start + t + 1);
       if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), (t >> 1) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[BN];
+      uint32_t sr[HALF];
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
-        tmem_ld32(tmem + lane_off + (b ? C::TM_S1 : C::TM_S0) + c * 32,
-                  *reinterpret_cast<uint32_t(*)[32]>(sr + c * 32));
+      for (int q = 0; q < HALF / 32; ++q)
+        tmem_ld32(tmem + lane_off + (b ? C::TM_S1 : C::TM_S0) + hf * HALF + q * 32,
+                  *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_s_free(b));
 
-      const int32_t j = __ldg(p.col_idx + start + t);
-      const int64_t valid = p.n_valid - int64_t(j) * BN;   // keys of this block that are real
-      float x[BN];
-      float mx = -INFINITY;
+      // Real keys of this half (only the block holding the sequence end is partial).
+      const int64_t valid = p.n_valid - int64_t(j) * BN - hf * HALF;
+      float mx;
+      if (valid >= HALF) {
+        // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (four partial chains)
+        float m4[4];
+        if (c >= 0.f) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        x[c] = (c < valid) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-        mx = fmaxf(mx, x[c]);
+          for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
+#pragma unroll
+          for (int e = 0; e < HALF; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sr[e]));
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) m4[e] = INFINITY;
+#pragma unroll
+          for (int e = 0; e < HALF; ++e) m4[e & 3] = fminf(m4[e & 3], __uint_as_float(sr[e]));
+          mx = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3])) * c;
+        }
+      } else {
+        mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < HALF; ++e)
+          if (e < valid) mx = fmaxf(mx, __uint_as_float(sr[e]) * c);
       }
+      // Row max over both halves.
+      {
+        bool good;
+        const float other = pair_exchange(t, mx, good);
+        if (!good) { ok = false; break; }
+        mx = fmaxf(mx, other);
+      }
+
       const float m_old = m_ref;
       if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
       const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float rs = 0.f;
-      uint32_t pk[BN / 2];
+      float r4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[HALF / 2];
+      if (valid >= HALF) {
 #pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        const float p0 = ex2_approx(x[c] - m_use), p1 = ex2_approx(x[c + 1] - m_use);
-        rs += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < HALF; e += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use));
+          r4[(e >> 1) & 3] += p0 + p1;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < HALF; e += 2) {
+          const float p0 = e < valid ? ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use)) : 0.f;
+          const float p1 = e + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use)) : 0.f;
+          r4[(e >> 1) & 3] += p0 + p1;
+          pk[e / 2] = pack_bf16x2(p0, p1);
+        }
       }
-      l = l * alpha + rs;
+      l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
 
       // P and O belong to the previous P*V product until it has completed.
       if (t >= 1) {
@@ -271,21 +358,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int q = 0; q < DH / 32; ++q) {
             uint32_t ov[32];
-            tmem_ld32(tmem + lane_off + C::TM_O + c * 32, ov);
+            tmem_ld32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tmem + lane_off + C::TM_O + c * 32, ov);
+            tmem_st32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
           }
           tmem_wait_st();
         }
       }
-      // P row -> shared memory, 128-byte swizzled K-major tile (64 keys per 128-byte slice).
+      // P half row -> shared memory, 128-byte swizzled K-major tile (64 keys per slice).
 #pragma unroll
-      for (int c8 = 0; c8 < BN / 8; ++c8) {
-        const int box = c8 >> 3, chunk = c8 & 7;
+      for (int c8 = 0; c8 < HALF / 8; ++c8) {
+        const int key8 = hf * (HALF / 8) + c8;    // 8-key chunk index within the row
+        const int box = key8 >> 3, chunk = key8 & 7;
         const uint32_t addr = sP + box * (BM * 128) + row * 128 + ((chunk ^ (row & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[c8 * 4]),
                      "r"(pk[c8 * 4 + 1]), "r"(pk[c8 * 4 + 2]), "r"(pk[c8 * 4 + 3])
@@ -303,16 +391,24 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       else tc_fence_after();
     }
     if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 3); }
+    // Row sum over both halves (exchange number n, after the n row-max exchanges).
+    float l_row = l;
+    if (ok && n > 0) {
+      bool good;
+      const float other = pair_exchange(n, l, good);
+      if (!good) { ok = false; *abort_flag = 1; report_fault(p.err, 5, 4); }
+      l_row += other;
+    }
     const int64_t grow = int64_t(i) * BN + row;           // row within the plane
     const bool store = row < BN && grow < p.n_pad;
-    const bool have = ok && n > 0 && l > 0.f;
-    const float inv_l = have ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = p.o + (plane * p.n_pad + grow) * D;
+    const bool have = ok && n > 0 && l_row > 0.f;
+    const float inv_l = have ? 1.f / l_row : 0.f;
+    __nv_bfloat16* orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int q = 0; q < DH / 32; ++q) {
       uint32_t ov[32];
       if (ok && n > 0) {
-        tmem_ld32(tmem + lane_off + C::TM_O + c * 32, ov);
+        tmem_ld32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
         tmem_wait_ld();
       }
       uint32_t w[16];
@@ -320,12 +416,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       for (int e = 0; e < 16; ++e)
         w[e] = have ? pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l) : 0u;
       if (store) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+        uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
         for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
       }
     }
-    if (store) p.lse[plane * p.n_pad + grow] = have ? (m_ref + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+    if (store && hf == 0)
+      p.lse[plane * p.n_pad + grow] = have ? (m_ref + __log2f(l_row)) * 0.69314718055994530942f : -INFINITY;
   }
 
   tc_fence_before();
