@@ -7,20 +7,24 @@
 // technical summary section 2) -- with an online softmax, so the cost is proportional to
 // the number of listed blocks.
 //
+// The listed key blocks are split between two softmax groups: group g takes the blocks at
+// list positions g, g+2, g+4, ... with its own S buffer, running max / sum, O accumulator
+// (all in TMEM) and P tile, and the two partial results are merged at the end.  The groups
+// run out of phase, so one group's exponentials (MUFU) overlap the other's max, P store
+// and waits, and the tensor core alternates between them.
+//
 // Warp roles (352 threads):
-//   warp 0      TMA producer: Q tile once, then K_j tiles into a 3-slot ring;
-//   warp 10     TMA producer: V_j tiles into a 2-slot ring;
-//   warp 1      MMA issuer (one thread): S = Q K_j^T into TMEM (two S buffers), and
-//               O += P V_j into a TMEM accumulator; owns the TMEM allocation;
-//   warps 2..9  softmax + epilogue, one (query row, column half) per thread (TMEM lane =
-//               row): read S from TMEM, update the running max (shared by the two halves
-//               of a row) and sum, write P (bf16) to shared memory in the tensor-core
-//               operand layout, rescale O in TMEM when the max moves by more than 2^8, and
-//               finally normalise O and write O and LSE.
+//   warp 0       TMA producer: Q tile once, then K_j tiles into a 3-slot ring;
+//   warp 10      TMA producer: V_j tiles into a 3-slot ring;
+//   warp 1       MMA issuer (one thread): S_g = Q K_j^T and O_g += P_g V_j (P_g read from
+//                TMEM, where it replaces S_g); owns TMEM;
+//   warps 2..5   softmax group 0, warps 6..9 softmax group 1: one query row per thread
+//                (TMEM lane = row); rescale O_g in TMEM only when the running max grows by
+//                more than 2^8; merge, normalise and store O and LSE at the end.
 //
 // Shared-memory operands use the 128-byte swizzle that TMA writes: a 64-element (128 B)
-// slice of each row, eight rows per 1024-byte atom.  Q, K and P are K-major; V is read
-// MN-major straight from its [keys, d] layout.
+// slice of each row, eight rows per 1024-byte atom.  Q and K are K-major; V is read
+// MN-major straight from its [keys, d] layout; P is the TMEM A operand of P*V.
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,9 +35,24 @@
 namespace lva {
 namespace {
 
+// Optional pipeline trace (compiled only with -DLVA_TRACE=<first CTA>): clock64 stamps of
+// pipeline events for kTraceCtas CTAs from the given one, slot = event * 64 + list position.
+#ifdef LVA_TRACE
+constexpr int kTraceCtas = 64, kTraceSlots = 32 * 64, kTraceBase = LVA_TRACE;
+__device__ unsigned long long g_trace[kTraceCtas][kTraceSlots];
+#define LVA_TRACE_AT(ev, t)                                                         \
+  do {                                                                              \
+    if (blockIdx.x >= kTraceBase && blockIdx.x < kTraceBase + kTraceCtas && (t) < 64) \
+      g_trace[blockIdx.x - kTraceBase][(ev) * 64 + (t)] = clock64();                   \
+  } while (0)
+#else
+#define LVA_TRACE_AT(ev, t) do { } while (0)
+#endif
+
 constexpr int BM = 128;            // query rows per MMA tile (TMEM lanes)
 constexpr int kSoftmaxWarp0 = 2;
-constexpr int kSoftmaxWarps = 8;   // two warps per TMEM lane quarter: one per column half
+constexpr int kGroupWarps = 4;     // one warp per TMEM lane quarter
+constexpr int kSoftmaxWarps = 2 * kGroupWarps;
 constexpr int kVWarp = kSoftmaxWarp0 + kSoftmaxWarps;   // V producer, after the softmax warps
 constexpr int kThreads = 32 * (kVWarp + 1);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when max grows > 2^8
@@ -53,30 +72,27 @@ struct AttnParams {
 
 template <int D, int BN>
 struct Cfg {
-  // K and V live in separate rings: a K slot is free once Q*K^T has read it, a V slot only
-  // after P*V, so K loads run further ahead than V loads.
-  static constexpr int KST = 3, VST = 2;
+  static constexpr int KST = 3, VST = 3;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + VST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2],
-  // s_free[2], p_full, o_done, final, pair[4 lane quarters][2 slots]
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], and per group
+  // s_full, p_full, o_done; final (MMA drain); merge (both groups' statistics)
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST, B_VE = B_VF + VST,
-                       B_SF = B_VE + VST, B_SE = B_SF + 2, B_P = B_SE + 2, B_O = B_P + 1,
-                       B_FIN = B_O + 1, B_PAIR = B_FIN + 1, NUM_BARS = B_PAIR + 8;
+                       B_SF = B_VE + VST, B_P = B_SF + 2, B_O = B_P + 2,
+                       B_FIN = B_O + 2, B_MERGE = B_FIN + 1, NUM_BARS = B_MERGE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  // row-max / row-sum exchange between the two column halves: [2 slots][2 halves][BM] floats
+  // per-row statistics of each group for the merge: [group][m, l][BM] floats
   static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
   // At least 120 KB so that one CTA (and one 512-column TMEM allocation) is resident per SM.
   static constexpr int SMEM_RAW = OFF_RED + 2 * 2 * BM * 4;
   static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
+  // S_g at column 128 g (P_g, bf16, overwrites its first BN/2 columns), O_g at 256 + 128 g
+  static constexpr uint32_t TM_S = 0, TM_O = 256;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
 };
@@ -113,20 +129,18 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     if (threadIdx.x == 0) report_fault(p.err, 4, 1023);
     return;
   }
-  const uint32_t sQ = s_base + C::OFF_Q, sK = s_base + C::OFF_K, sV = s_base + C::OFF_V,
-                 sP = s_base + C::OFF_P;
+  const uint32_t sQ = s_base + C::OFF_Q, sK = s_base + C::OFF_K, sV = s_base + C::OFF_V;
   const uint32_t bar0 = s_base + C::OFF_BAR;
   const uint32_t bar_q = bar0 + 8u * C::B_Q;
   auto bar_k_full = [&](int s) { return bar0 + 8u * (C::B_KF + s); };
   auto bar_k_empty = [&](int s) { return bar0 + 8u * (C::B_KE + s); };
   auto bar_v_full = [&](int s) { return bar0 + 8u * (C::B_VF + s); };
   auto bar_v_empty = [&](int s) { return bar0 + 8u * (C::B_VE + s); };
-  auto bar_s_full = [&](int b) { return bar0 + 8u * (C::B_SF + b); };
-  auto bar_s_free = [&](int b) { return bar0 + 8u * (C::B_SE + b); };
-  const uint32_t bar_p_full = bar0 + 8u * C::B_P;
-  const uint32_t bar_o_done = bar0 + 8u * C::B_O;
+  auto bar_s_full = [&](int g) { return bar0 + 8u * (C::B_SF + g); };
+  auto bar_p_full = [&](int g) { return bar0 + 8u * (C::B_P + g); };
+  auto bar_o_done = [&](int g) { return bar0 + 8u * (C::B_O + g); };
   const uint32_t bar_final = bar0 + 8u * C::B_FIN;
-  auto bar_pair = [&](int q, int slot) { return bar0 + 8u * (C::B_PAIR + 2 * q + slot); };
+  const uint32_t bar_merge = bar0 + 8u * C::B_MERGE;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   // Stays zero: the drain waits after an abort are bounded by time alone.
@@ -148,11 +162,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     mbar_init(bar_q, 1);
     for (int s = 0; s < C::KST; ++s) { mbar_init(bar_k_full(s), 1); mbar_init(bar_k_empty(s), 1); }
     for (int s = 0; s < C::VST; ++s) { mbar_init(bar_v_full(s), 1); mbar_init(bar_v_empty(s), 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(bar_s_full(b), 1); mbar_init(bar_s_free(b), kSoftmaxWarps); }
-    mbar_init(bar_p_full, kSoftmaxWarps);
-    mbar_init(bar_o_done, 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar_s_full(g), 1);
+      mbar_init(bar_p_full(g), kGroupWarps);
+      mbar_init(bar_o_done(g), 1);
+    }
     mbar_init(bar_final, 1);
-    for (int q = 0; q < 4; ++q) { mbar_init(bar_pair(q, 0), 2); mbar_init(bar_pair(q, 1), 2); }
+    mbar_init(bar_merge, kSoftmaxWarps);
     *abort_flag = 0;
     *never = 0;
     mbar_fence_init();
@@ -162,6 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) LVA_TRACE_AT(20, 0);
 
   // One TMA producer loop: tile t of `n` goes to slot t % ST of a ring whose slots are
   // released by `empty` barriers; after an abort, waits for the loads already issued.
@@ -175,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       const int32_t j = __ldg(p.col_idx + start + t);
       const int32_t kv_row = int32_t(plane * p.n_pad + int64_t(j) * BN);
       mbar_arrive_expect_tx(full0 + 8u * s, C::KV_BYTES);
+      LVA_TRACE_AT(code == 1 ? 14 : 15, t);
       for (int c = 0; c < D / 64; ++c)
         tma_load_2d(ring + s * C::KV_BYTES + c * BN * 128, tmap, c * 64, kv_row, full0 + 8u * s);
       issued = t + 1;
@@ -202,40 +220,47 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order: S(t) for group t&1, then O += P V for the block before it (other group).
+    // P_g lives in S_g's TMEM columns; the tensor core executes this thread's MMAs in
+    // order, so S(t+2) is written only after P(t) V has read P(t).
     if (lane == 0 && n > 0) {
+      // Descriptors are built once; an MMA only adds a byte offset / 16 to the start-address
+      // field (shared addresses stay below 2^18 bytes, so the 14-bit field never carries).
+      const uint64_t q_desc = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t k_desc = smem_desc_sw128(sK, 16, 1024);
+      const uint64_t v_desc = smem_desc_sw128(sV, BN * 128, 1024);
       bool ok = mbar_wait(bar_q, 0, abort_flag);
       bool any_mma = false;
       auto issue_pv = [&](int t) -> bool {
-        const int s = t % C::VST;
-        if (!mbar_wait(bar_p_full, t & 1, abort_flag)) return false;
+        const int g = t & 1, u = t >> 1, s = t % C::VST;
+        if (!mbar_wait(bar_p_full(g), u & 1, abort_flag)) return false;
         if (!mbar_wait(bar_v_full(s), (t / C::VST) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t v_base = sV + s * C::KV_BYTES;
+        LVA_TRACE_AT(1, t);
+        const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
+        const uint32_t o_tm = tmem + C::TM_O + 128 * g, p_tm = tmem + C::TM_S + 128 * g;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(sP + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
-          const uint64_t b = smem_desc_sw128(v_base + kk * 16 * 128, BN * 128, 1024);
-          umma_f16_ss(tmem + C::TM_O, a, b, C::IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_f16_ts(o_tm, p_tm + kk * 8, vs + uint64_t((kk * 16 * 128) >> 4), C::IDESC_PV,
+                      (u > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar_v_empty(s));
-        umma_commit(bar_o_done);
+        umma_commit(bar_o_done(g));
         return true;
       };
       for (int t = 0; ok && t < n; ++t) {
-        const int s = t % C::KST, b = t & 1;
+        const int s = t % C::KST, g = t & 1;
         ok = mbar_wait(bar_k_full(s), (t / C::KST) & 1, abort_flag);
-        if (ok && t >= 2) ok = mbar_wait(bar_s_free(b), ((t >> 1) - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t k_base = sK + s * C::KV_BYTES;
-        const uint32_t s_tm = tmem + (b ? C::TM_S1 : C::TM_S0);
+        LVA_TRACE_AT(0, t);
+        const uint64_t ks = k_desc + uint64_t((s * C::KV_BYTES) >> 4);
+        const uint32_t s_tm = tmem + C::TM_S + 128 * g;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = smem_desc_sw128(sQ + (kk / 4) * BM * 128 + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(k_base + (kk / 4) * BN * 128 + (kk % 4) * 32, 16, 1024);
-          umma_f16_ss(s_tm, a, bd, C::IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(bar_s_full(b));
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_f16_ss(s_tm, q_desc + uint64_t(((kk / 4) * BM * 128 + (kk % 4) * 32) >> 4),
+                      ks + uint64_t(((kk / 4) * BN * 128 + (kk % 4) * 32) >> 4), C::IDESC_QK,
+                      kk > 0 ? 1u : 0u);
+        umma_commit(bar_s_full(g));
         umma_commit(bar_k_empty(s));
         any_mma = true;
         if (t >= 1) ok = issue_pv(t - 1);
@@ -249,93 +274,70 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax + epilogue
-    // Thread = (query row, column half).  Warps w and w+4 share a TMEM lane quarter, so
-    // they own the same 32 rows; the first takes key/O columns [0, half), the second
-    // [half, 2*half).  They exchange the row max once per key block.
-    constexpr int HALF = BN / 2, DH = D / 2;
-    const int sw = warp - kSoftmaxWarp0;          // 0..7
-    const int hf = sw >> 2;                       // column half
+    // ------------------------------------------------------------ softmax groups + epilogue
+    const int g = (warp - kSoftmaxWarp0) / kGroupWarps;   // group: list positions g, g+2, ...
     const int sub = warp & 3;                     // TMEM lane quarter this warp may access
     const int row = sub * 32 + lane;              // row of the 128-row tile
     const uint32_t lane_off = uint32_t(sub * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);   // [slot][half][row]
-    // Exchange of one value per row with the partner warp (other column half).  Exchange
-    // number `seq` uses slot seq & 1; the partner's read of a slot always precedes its
-    // arrival on the next exchange, so a slot is never overwritten before it is read.
-    auto pair_exchange = [&](int seq, float v, bool& good) -> float {
-      float* slot = red + (seq & 1) * 2 * BM;
-      slot[hf * BM + row] = v;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pair(sub, seq & 1));
-      good = __all_sync(0xffffffffu, mbar_wait(bar_pair(sub, seq & 1), (seq >> 1) & 1, abort_flag));
-      return good ? slot[(1 - hf) * BM + row] : 0.f;
-    };
+    const uint32_t tS = tmem + lane_off + C::TM_S + 128 * g;
+    const uint32_t tO = tmem + lane_off + C::TM_O + 128 * g;
     const float c = p.scale_log2;                 // scores -> log2 units
+    const int ng = n > g ? (n - g + 1) / 2 : 0;   // blocks of this group
     float m_ref = -INFINITY;                      // running max in log2 units (lazy)
-    float l = 0.f;                                // this half's share of the row sum
+    float l = 0.f;
     bool ok = true;
     if (bad && threadIdx.x == kSoftmaxWarp0 * 32) report_fault(p.err, 1, int(csr & 0x7fffffff));
-    int32_t jn = n > 0 ? __ldg(p.col_idx + start) : 0;
+    int32_t jn = ng > 0 ? __ldg(p.col_idx + start + g) : 0;
 
-    for (int t = 0; t < n; ++t) {
-      const int b = t & 1;
+    const bool tr = (sub == 2 && lane == 0);     // first warp of the group traces
+    for (int u = 0; u < ng; ++u) {
+      const int t = 2 * u + g;
       const int32_t j = jn;
-      if (t + 1 < n) jn = __ldg(p.col_idx + start + t + 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), (t >> 1) & 1, abort_flag))) { ok = false; break; }
+      if (u + 1 < ng) jn = __ldg(p.col_idx + start + t + 2);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(g), u & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[HALF];
+      if (tr) LVA_TRACE_AT(2 + 6 * g, t);
+      uint32_t sr[BN];
 #pragma unroll
-      for (int q = 0; q < HALF / 32; ++q)
-        tmem_ld32(tmem + lane_off + (b ? C::TM_S1 : C::TM_S0) + hf * HALF + q * 32,
-                  *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
+      for (int q = 0; q < BN / 32; ++q)
+        tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_s_free(b));
+      if (tr) LVA_TRACE_AT(3 + 6 * g, t);
 
-      // Real keys of this half (only the block holding the sequence end is partial).
-      const int64_t valid = p.n_valid - int64_t(j) * BN - hf * HALF;
+      // Real keys of this block (only the block holding the sequence end is partial).
+      const int64_t valid = p.n_valid - int64_t(j) * BN;
       float mx;
-      if (valid >= HALF) {
+      if (valid >= BN) {
         // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (four partial chains)
         float m4[4];
         if (c >= 0.f) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < HALF; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sr[e]));
+          for (int e = 0; e < BN; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sr[e]));
           mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
         } else {
 #pragma unroll
           for (int e = 0; e < 4; ++e) m4[e] = INFINITY;
 #pragma unroll
-          for (int e = 0; e < HALF; ++e) m4[e & 3] = fminf(m4[e & 3], __uint_as_float(sr[e]));
+          for (int e = 0; e < BN; ++e) m4[e & 3] = fminf(m4[e & 3], __uint_as_float(sr[e]));
           mx = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3])) * c;
         }
       } else {
         mx = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < HALF; ++e)
+        for (int e = 0; e < BN; ++e)
           if (e < valid) mx = fmaxf(mx, __uint_as_float(sr[e]) * c);
       }
-      // Row max over both halves.
-      {
-        bool good;
-        const float other = pair_exchange(t, mx, good);
-        if (!good) { ok = false; break; }
-        mx = fmaxf(mx, other);
-      }
-
       const float m_old = m_ref;
       if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
       const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       float r4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[HALF / 2];
-      if (valid >= HALF) {
+      uint32_t pk[BN / 2];
+      if (valid >= BN) {
 #pragma unroll
-        for (int e = 0; e < HALF; e += 2) {
+        for (int e = 0; e < BN; e += 2) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use));
           const float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use));
           r4[(e >> 1) & 3] += p0 + p1;
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < HALF; e += 2) {
+        for (int e = 0; e < BN; e += 2) {
           const float p0 = e < valid ? ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use)) : 0.f;
           const float p1 = e + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use)) : 0.f;
           r4[(e >> 1) & 3] += p0 + p1;
@@ -351,78 +353,93 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         }
       }
       l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
+      if (tr) LVA_TRACE_AT(4 + 6 * g, t);
 
-      // P and O belong to the previous P*V product until it has completed.
-      if (t >= 1) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (t - 1) & 1, abort_flag))) { ok = false; break; }
+      // O_g may be rescaled only after this group's previous P*V has completed; without a
+      // rescale the next P*V simply follows it on the tensor pipe.
+      if (u >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(g), (u - 1) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        if (tr) LVA_TRACE_AT(5 + 6 * g, t);
 #pragma unroll 1
-          for (int q = 0; q < DH / 32; ++q) {
-            uint32_t ov[32];
-            tmem_ld32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
-            tmem_wait_ld();
+        for (int q = 0; q < D / 32; ++q) {
+          uint32_t ov[32];
+          tmem_ld32(tO + q * 32, ov);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(tO + q * 32, ov);
         }
       }
-      // P half row -> shared memory, 128-byte swizzled K-major tile (64 keys per slice).
+      // P row (bf16 pairs) -> TMEM over the first BN/2 columns of S_g, the A operand of P*V.
 #pragma unroll
-      for (int c8 = 0; c8 < HALF / 8; ++c8) {
-        const int key8 = hf * (HALF / 8) + c8;    // 8-key chunk index within the row
-        const int box = key8 >> 3, chunk = key8 & 7;
-        const uint32_t addr = sP + box * (BM * 128) + row * 128 + ((chunk ^ (row & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[c8 * 4]),
-                     "r"(pk[c8 * 4 + 1]), "r"(pk[c8 * 4 + 2]), "r"(pk[c8 * 4 + 3])
-                     : "memory");
-      }
-      fence_proxy_async_smem();
+      for (int q = 0; q < BN / 64; ++q)
+        tmem_st32(tS + q * 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + q * 32));
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p_full);
+      if (lane == 0) mbar_arrive(bar_p_full(g));
+      if (tr) LVA_TRACE_AT(7 + 6 * g, t);
     }
 
-    // ------------------------------------------------------------ epilogue
-    if (ok && n > 0) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (n - 1) & 1, abort_flag))) ok = false;
+    // ------------------------------------------------------------ merge + epilogue
+    if (tr) LVA_TRACE_AT(16 + g, 0);
+    if (ok && ng > 0) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(g), (ng - 1) & 1, abort_flag))) ok = false;
       else tc_fence_after();
     }
     if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 3); }
-    // Row sum over both halves (exchange number n, after the n row-max exchanges).
-    float l_row = l;
-    if (ok && n > 0) {
-      bool good;
-      const float other = pair_exchange(n, l, good);
-      if (!good) { ok = false; *abort_flag = 1; report_fault(p.err, 5, 4); }
-      l_row += other;
+    // Publish this group's (max, sum) per row; read the other group's.
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);      // [group][m, l][row]
+    red[(2 * g) * BM + row] = m_ref;
+    red[(2 * g + 1) * BM + row] = ok ? l : 0.f;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_merge);
+    if (!__all_sync(0xffffffffu, mbar_wait(bar_merge, 0, abort_flag))) {
+      ok = false; *abort_flag = 1; report_fault(p.err, 5, 4);
     }
+    float m0 = red[0 * BM + row], l0 = red[1 * BM + row];
+    float m1 = red[2 * BM + row], l1 = red[3 * BM + row];
+    if (!ok) { l0 = 0.f; l1 = 0.f; }
+    const float m = fmaxf(m0, m1);
+    const float a0 = l0 > 0.f ? ex2_approx(m0 - m) : 0.f;     // weights of the two partials
+    const float a1 = l1 > 0.f ? ex2_approx(m1 - m) : 0.f;
+    const float lt = a0 * l0 + a1 * l1;
+    const bool have = lt > 0.f;
+    const float w0 = have ? a0 / lt : 0.f, w1 = have ? a1 / lt : 0.f;
+    const bool use0 = ok && n > 0 && l0 > 0.f, use1 = ok && n > 1 && l1 > 0.f;
+
+    // Each group normalises and stores half of the O columns of its rows.
+    constexpr int DH = D / 2;
     const int64_t grow = int64_t(i) * BN + row;           // row within the plane
     const bool store = row < BN && grow < p.n_pad;
-    const bool have = ok && n > 0 && l_row > 0.f;
-    const float inv_l = have ? 1.f / l_row : 0.f;
-    __nv_bfloat16* orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
+    __nv_bfloat16* orow = p.o + (plane * p.n_pad + grow) * D + g * DH;
+    const uint32_t tO0 = tmem + lane_off + C::TM_O + g * DH, tO1 = tO0 + 128;
 #pragma unroll 1
     for (int q = 0; q < DH / 32; ++q) {
-      uint32_t ov[32];
+      uint32_t o0[32], o1[32];
       if (ok && n > 0) {
-        tmem_ld32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
+        tmem_ld32(tO0 + q * 32, o0);
+        if (n > 1) tmem_ld32(tO1 + q * 32, o1);
         tmem_wait_ld();
       }
       uint32_t w[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        w[e] = have ? pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l) : 0u;
+      for (int e = 0; e < 16; ++e) {
+        float x0 = 0.f, x1 = 0.f;
+        if (use0) { x0 = __uint_as_float(o0[2 * e]) * w0; x1 = __uint_as_float(o0[2 * e + 1]) * w0; }
+        if (use1) { x0 += __uint_as_float(o1[2 * e]) * w1; x1 += __uint_as_float(o1[2 * e + 1]) * w1; }
+        w[e] = pack_bf16x2(x0, x1);
+      }
       if (store) {
         uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
         for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
       }
     }
-    if (store && hf == 0)
-      p.lse[plane * p.n_pad + grow] = have ? (m_ref + __log2f(l_row)) * 0.69314718055994530942f : -INFINITY;
+    if (tr) LVA_TRACE_AT(18 + g, 0);
+    if (store && g == 0)
+      p.lse[plane * p.n_pad + grow] = have ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
   }
 
   tc_fence_before();
@@ -502,6 +519,12 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
 }
 
 }  // namespace
+
+#ifdef LVA_TRACE
+extern "C" int lva_trace_copy(void* dst, size_t bytes) {
+  return int(cudaMemcpyFromSymbol(dst, g_trace, bytes < sizeof(g_trace) ? bytes : sizeof(g_trace)));
+}
+#endif
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why) {
   if (a.d == 128 && a.block_size == 128) return launch_cfg<128, 128>(a, stream, why);
