@@ -356,6 +356,98 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _time_cuda(fn, reps=7, warmup=2):
+    """Median ms of `fn` over `reps` launches (CUDA events on the current stream)."""
+    for _ in range(warmup):
+        fn()
+    ts = []
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b))
+    return float(np.median(ts))
+
+
+def run_report(args):
+    """One JSON line per (workload, mask): attention ms / TFLOP/s / fraction of peak, reorder
+    and mask-build GB/s; then the density sweep fit time = a + b * active pairs."""
+    import block_sparse_attention_lva_b200 as lva
+    from synthetic import static_calibrated_mask
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    burst, sustained, hbm, peak_kind = _peaks()
+    names = args.report.split(",")
+    for name in names:
+        if name == "stress":
+            continue
+        w = WORKLOADS[name]
+        q, k, v = make_qkv(w)
+        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        del q, k, v
+        sweep = []
+        for spec in mask_variants(w):
+            static = static_calibrated_mask(w) if spec["kind"] == "static" else None
+            layer = lva.VideoBlockSparseAttention(w.B, w.H, w.d, (w.T, w.Hg, w.Wg), w.tile, w.block_size, spec,
+                                                  static_mask=static, scale=w.scale, device=dev)
+            layer(qd, kd, vd, step=0)
+            torch.cuda.synchronize()
+            nnz = int(layer.nnz.item())
+            pairs = nnz * (w.B * w.H if layer.mask_heads == 1 else w.B)
+            flops = pairs * _flops_per_nnz(w)
+            ms = _time_cuda(layer.attend)
+            layer._built_step = None
+            ms_mask = _time_cuda(lambda: (setattr(layer, "_built_step", None), layer.build_mask(0)))
+            mask_bytes = (layer.mask_heads * w.nb * w.nb if spec["kind"] == "static" else 0) \
+                + 4 * (layer.mask_heads * w.nb + 1) + 4 * nnz
+            ms_reorder = _time_cuda(lambda: lva.lva_reorder_tokens(
+                qd.view(w.B * w.H, w.n_valid, w.d), layer.q_t.view(w.B * w.H, w.n_pad, w.d),
+                (w.T, w.Hg, w.Wg), w.tile, w.n_pad))
+            reorder_bytes = w.B * w.H * (w.n_valid + w.n_pad) * w.d * 2
+            status, detail = lva.lva_device_error()
+            line = {"report": name, "mask": spec["label"], "active_pairs": pairs,
+                    "density": nnz / (layer.mask_heads * w.nb * w.nb), "attn_ms": ms,
+                    "tflops": flops / ms / 1e9, "frac_of_sustained": flops / ms / 1e9 / sustained,
+                    "frac_of_burst": flops / ms / 1e9 / burst, "mask_build_us": ms_mask * 1e3,
+                    "mask_gbs": mask_bytes / ms_mask / 1e6, "reorder_ms": ms_reorder,
+                    "reorder_gbs": reorder_bytes / ms_reorder / 1e6, "hbm_peak_gbs": hbm,
+                    "peak_kind": peak_kind, "kernel_error": status}
+            print(json.dumps(line), flush=True)
+            if spec["kind"] in ("window_anchor", "all"):
+                sweep.append((pairs, ms, nnz / (layer.mask_heads * w.nb * w.nb)))
+            del layer
+            torch.cuda.empty_cache()
+        if len(sweep) >= 3:
+            x = np.array([p for p, _, _ in sweep], dtype=np.float64)
+            y = np.array([m for _, m, _ in sweep], dtype=np.float64)
+            A = np.stack([np.ones_like(x), x], axis=1)
+            (a, b), *_ = np.linalg.lstsq(A, y, rcond=None)
+            r2 = 1 - np.sum((y - (a + b * x)) ** 2) / np.sum((y - y.mean()) ** 2)
+            d = np.array([dd for _, _, dd in sweep])
+            i10 = int(np.argmin(np.abs(d - 0.10)))
+            print(json.dumps({"report": name, "density_sweep": [{"density": float(dd), "ms": float(m)} for _, m, dd in sweep],
+                              "fit_ms": {"intercept": float(a), "per_pair_us": float(b * 1e3), "r2": float(r2),
+                                         "intercept_share_of_10pct": float(a / y[i10])}}), flush=True)
+        del qd, kd, vd
+        torch.cuda.empty_cache()
+    # mask-builder stress size: static mask, 40 heads x 4096 x 4096 blocks (671 MB read)
+    if "stress" in names or args.report_stress:
+        hm, nb = 40, 4096
+        g = torch.Generator(device=dev).manual_seed(5)
+        dense = (torch.rand((hm, nb, nb), generator=g, device=dev) < 0.3).to(torch.uint8)
+        params = lva.MaskParams(lva.LVA_MASK_STATIC, nb * 128, nb * 128, 128, hm)
+        row_ptr = torch.empty(hm * nb + 1, dtype=torch.int32, device=dev)
+        col_idx = torch.empty(lva.lva_block_mask_max_nnz(params), dtype=torch.int32, device=dev)
+        nnz = torch.empty(1, dtype=torch.int32, device=dev)
+        ms = _time_cuda(lambda: lva.lva_build_block_mask(params, dense, row_ptr, col_idx, nnz))
+        n = int(nnz.item())
+        byts = hm * nb * nb + 4 * (hm * nb + 1) + 4 * n
+        print(json.dumps({"report": "mask_stress", "mask_heads": hm, "nb": nb, "nnz": n, "ms": ms,
+                          "gbs": byts / ms / 1e6, "hbm_peak_gbs": hbm}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -365,10 +457,15 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--report", default="", help="comma list of workloads (tiny,small,static,large,long,stress): "
+                    "per-mask kernel timings and the density sweep fit instead of the bench line")
+    ap.add_argument("--report-stress", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.report:
+        run_report(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_lva(args)
