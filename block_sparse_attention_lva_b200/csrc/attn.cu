@@ -308,19 +308,21 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       const int64_t valid = p.n_valid - int64_t(j) * BN;
       float mx;
       if (valid >= BN) {
-        // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (four partial chains)
+        // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (3-input max, 4 chains)
         float m4[4];
         if (c >= 0.f) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < BN; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sr[e]));
+          for (int e = 0; e < BN / 2; ++e)
+            m4[e & 3] = fmax3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
           mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
         } else {
 #pragma unroll
           for (int e = 0; e < 4; ++e) m4[e] = INFINITY;
 #pragma unroll
-          for (int e = 0; e < BN; ++e) m4[e & 3] = fminf(m4[e & 3], __uint_as_float(sr[e]));
+          for (int e = 0; e < BN / 2; ++e)
+            m4[e & 3] = fmin3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
           mx = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3])) * c;
         }
       } else {
@@ -336,13 +338,30 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       float r4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[BN / 2];
       if (valid >= BN) {
+        // Pairs of elements with packed fp32 math; every third pair takes its exponentials
+        // on the FMA pipe, the rest on the MUFU, which balances the two units.
+        const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
+        uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
-        for (int e = 0; e < BN; e += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use));
-          r4[(e >> 1) & 3] += p0 + p1;
-          pk[e / 2] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < BN / 2; ++e) {
+          const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
+          uint64_t p2;
+          if (e % 3 == 2) {
+            p2 = exp2_poly_f2(x2);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          acc[e & 1] = f2_add(acc[e & 1], p2);
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
+          pk[e] = pack_bf16x2(p0, p1);
         }
+        float a0, a1, b0, b1;
+        f2_unpack(acc[0], a0, a1);
+        f2_unpack(acc[1], b0, b1);
+        r4[0] = a0; r4[1] = a1; r4[2] = b0; r4[3] = b1;
       } else {
 #pragma unroll
         for (int e = 0; e < BN; e += 2) {
