@@ -63,9 +63,10 @@ class VideoBlockSparseAttention:
             raise ValueError(f"invalid mask parameters {self.params}")
         kw = dict(device=self.device)
         shape = (B, H, self.n_pad, d)
-        self.q_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
-        self.k_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
-        self.v_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
+        # Q, K, V in tile order share one buffer so that a stacked raster QKV is reordered
+        # by a single launch.
+        self.qkv_t = torch.empty((3,) + shape, dtype=torch.bfloat16, **kw)
+        self.q_t, self.k_t, self.v_t = self.qkv_t[0], self.qkv_t[1], self.qkv_t[2]
         self.o_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
         self.lse = torch.empty((B, H, self.n_pad), dtype=torch.float32, **kw)
         self.o = torch.empty((B, H, self.n_valid, d), dtype=torch.bfloat16, **kw)
@@ -84,8 +85,23 @@ class VideoBlockSparseAttention:
         lb.lva_build_block_mask(self.params, self.dense_mask, self.row_ptr, self.col_idx, self.nnz)
         self._built_step = key
 
+    @staticmethod
+    def _stacked(q, k, v):
+        """True when q, k, v are consecutive, equally sized, contiguous slices of one buffer."""
+        if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+            return False
+        nbytes = q.numel() * q.element_size()
+        return (k.data_ptr() == q.data_ptr() + nbytes and v.data_ptr() == k.data_ptr() + nbytes
+                and q.shape == k.shape == v.shape and q.dtype == k.dtype == v.dtype)
+
     def reorder_in(self, q, k, v):
         P = self.B * self.H
+        if self._stacked(q, k, v):
+            base = q.view(-1)
+            src = torch.as_strided(base, (3 * P, self.n_valid, self.d), (self.n_valid * self.d, self.d, 1))
+            lb.lva_reorder_tokens(src, self.qkv_t.view(3 * P, self.n_pad, self.d), self.grid, self.tile,
+                                  self.n_pad, inverse=False)
+            return
         for src, dst in ((q, self.q_t), (k, self.k_t), (v, self.v_t)):
             lb.lva_reorder_tokens(src.view(P, self.n_valid, self.d), dst.view(P, self.n_pad, self.d),
                                   self.grid, self.tile, self.n_pad, inverse=False)

@@ -68,6 +68,26 @@ def test_against_oracle_full(B, H, n_pad, n_valid, d, bs, hm, density, seed):
     check_o_lse(o, lse, o_ref, lse_ref, f"shape {(B, H, n_pad, d, bs)}")
 
 
+def test_many_items_mixed_rows():
+    # 2 x 8 heads x 32 query blocks = 512 work items (more than one wave of CTAs), per-head
+    # masks with empty rows, single-block rows and full rows interleaved.
+    B, H, n_pad, d, bs = 2, 8, 4096, 128, 128
+    n_valid = 4000
+    q = _rand_bf16((B, H, n_pad, d), 71)
+    k = _rand_bf16((B, H, n_pad, d), 72)
+    v = _rand_bf16((B, H, n_pad, d), 73)
+    nb = n_pad // bs
+    rng = np.random.default_rng(7)
+    masks = rng.random((H, nb, nb)) < rng.random((H, nb, 1))        # row densities 0..1
+    masks[:, ::7] = False                                            # empty rows
+    masks[:, 3::11] = False
+    masks[:, 3::11, 5] = True                                        # one block only
+    masks[:, 1::13] = True                                           # full rows
+    o, lse = _attn_gpu(q, k, v, masks, bs, n_valid, 1.0 / math.sqrt(d))
+    o_ref, lse_ref = attention_blocked(q, k, v, masks, bs, n_valid, 1.0 / math.sqrt(d))
+    check_o_lse(o, lse, o_ref, lse_ref, "many items")
+
+
 def test_tiny_workload():
     w = WORKLOADS["tiny"]
     spec = mask_variants(w)[0]

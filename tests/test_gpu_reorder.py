@@ -62,3 +62,20 @@ def test_iota_returns_permutation():
     got = out.view(torch.int32).cpu().numpy()[0, :, 0]
     perm = tile_permutation(w.T, w.Hg, w.Wg, *w.tile)
     assert np.array_equal(got[:n], perm) and np.all(got[n:] == 0)
+
+
+def test_stacked_qkv_single_launch_matches_separate():
+    import block_sparse_attention_lva_b200 as lva
+    dev = require_gpu()
+    w = WORKLOADS["small"]
+    g = torch.Generator().manual_seed(3)
+    qkv = torch.randint(-2**15, 2**15, (3, 1, 4, w.n_valid, w.d), generator=g, dtype=torch.int32)
+    qkv = qkv.to(torch.int16).view(torch.bfloat16).to(dev)
+    spec = dict(kind="all")
+    a = lva.VideoBlockSparseAttention(1, 4, w.d, (w.T, w.Hg, w.Wg), w.tile, w.block_size, spec, device=dev)
+    b = lva.VideoBlockSparseAttention(1, 4, w.d, (w.T, w.Hg, w.Wg), w.tile, w.block_size, spec, device=dev)
+    assert a._stacked(qkv[0], qkv[1], qkv[2])
+    a.reorder_in(qkv[0], qkv[1], qkv[2])                            # one launch over 3 * B * H planes
+    b.reorder_in(qkv[0].clone(), qkv[1].clone(), qkv[2].clone())    # three launches
+    torch.cuda.synchronize()
+    assert torch.equal(a.qkv_t.view(torch.int16), b.qkv_t.view(torch.int16))
