@@ -19,6 +19,7 @@ LVA_MASK_WINDOW_ANCHOR = 0
 LVA_MASK_STATIC = 1
 LVA_MASK_ALL = 2
 LVA_MASK_TWO_STAGE = 3
+LVA_MASK_LVSA_FRAMES = 4
 
 STATUS_NAMES = {0: "LVA_OK", 1: "LVA_ERR_INVALID_ARG", 2: "LVA_ERR_UNSUPPORTED",
                 3: "LVA_ERR_CAPACITY", 4: "LVA_ERR_CUDA", 5: "LVA_ERR_TIMEOUT"}
@@ -32,7 +33,8 @@ class LvaMaskParams(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("mask_heads", ctypes.c_int), ("block_size", ctypes.c_int),
                 ("n_pad", ctypes.c_int64), ("n_valid", ctypes.c_int64),
                 ("window_unit_tokens", ctypes.c_int64), ("window_radius", ctypes.c_int),
-                ("num_anchors", ctypes.c_int), ("step", ctypes.c_int), ("group_blocks", ctypes.c_int)]
+                ("num_anchors", ctypes.c_int), ("step", ctypes.c_int), ("group_blocks", ctypes.c_int),
+                ("budget_frames", ctypes.c_int)]
 
 
 SIGNATURES = {
@@ -113,11 +115,12 @@ class MaskParams:
     num_anchors: int = 0
     step: int = 0
     group_blocks: int = 1
+    budget_frames: int = 1
 
     def to_c(self) -> LvaMaskParams:
         return LvaMaskParams(self.kind, self.mask_heads, self.block_size, self.n_pad, self.n_valid,
                              self.window_unit_tokens, self.window_radius, self.num_anchors, self.step,
-                             self.group_blocks)
+                             self.group_blocks, self.budget_frames)
 
 
 def lva_version() -> int:

@@ -120,6 +120,14 @@ static lva_status check_mask_params(const lva_mask_params* p) {
     case LVA_MASK_ALL:
       if (p->mask_heads != 1) return fail(LVA_ERR_INVALID_ARG, "mask: parametric kinds build one mask head");
       break;
+    case LVA_MASK_LVSA_FRAMES: {
+      if (p->window_unit_tokens < 1 || p->num_anchors < 0 || p->step < 0 || p->budget_frames < 1)
+        return fail(LVA_ERR_INVALID_ARG, "mask: LVSA frames need unit >= 1, anchors >= 0, step >= 0, budget >= 1");
+      const int64_t frames = (p->n_valid + p->window_unit_tokens - 1) / p->window_unit_tokens;
+      if (p->num_anchors > frames) return fail(LVA_ERR_INVALID_ARG, "mask: more global frames than frames");
+      if (p->mask_heads != 1) return fail(LVA_ERR_INVALID_ARG, "mask: parametric kinds build one mask head");
+      break;
+    }
     case LVA_MASK_STATIC:
       break;
     default:
@@ -159,6 +167,7 @@ lva_status lva_build_block_mask(const lva_mask_params* p, const uint8_t* dense_m
   a.num_anchors = p->num_anchors;
   a.step = p->step;
   a.group_blocks = p->group_blocks;
+  a.budget_frames = p->budget_frames;
   a.dense = dense_mask;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;

@@ -25,7 +25,7 @@ struct MaskArgs {
   int block_size;
   int64_t n_pad, n_valid;
   int64_t unit_tokens;
-  int radius, num_anchors, step, group_blocks;
+  int radius, num_anchors, step, group_blocks, budget_frames;
   const uint8_t* dense;
   int32_t* row_ptr;
   int32_t* col_idx;

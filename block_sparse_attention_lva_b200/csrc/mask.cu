@@ -14,7 +14,7 @@
 namespace lva {
 namespace {
 
-enum Kind { kWindowAnchor = 0, kStatic = 1, kAll = 2, kTwoStage = 3 };
+enum Kind { kWindowAnchor = 0, kStatic = 1, kAll = 2, kTwoStage = 3, kLvsaFrames = 4 };
 
 struct MaskDev {
   int kind;
@@ -24,6 +24,7 @@ struct MaskDev {
   int64_t radius;
   int64_t anchors, step;
   int64_t group;
+  int64_t frames, budget;   // LVSA frames: T and C
   const uint8_t* dense;
 };
 
@@ -39,13 +40,35 @@ __device__ __forceinline__ void block_units(const MaskDev& m, int64_t i, int64_t
   }
 }
 
-// Is key block j one of the anchors {(floor(a*nb/G) + s) mod nb : a < G}?
+// Is x one of the anchors {(floor(a*n/G) + s) mod n : a < G}?  (n = blocks or frames)
+__device__ __forceinline__ bool is_anchor_of(int64_t x, int64_t n, int64_t G, int64_t s) {
+  if (G <= 0) return false;
+  const int64_t xx = ((x - s) % n + n) % n;
+  // smallest a with floor(a*n/G) >= xx is ceil(xx*G/n)
+  const int64_t a = (xx * G + n - 1) / n;
+  return a < G && (a * n) / G == xx;
+}
+
 __device__ __forceinline__ bool is_anchor(const MaskDev& m, int64_t j) {
-  if (m.anchors <= 0) return false;
-  const int64_t jj = ((j - m.step) % m.nb + m.nb) % m.nb;
-  // smallest a with floor(a*nb/G) >= jj is ceil(jj*G/nb)
-  const int64_t a = (jj * m.anchors + m.nb - 1) / m.nb;
-  return a < m.anchors && (a * m.nb) / m.anchors == jj;
+  return is_anchor_of(j, m.nb, m.anchors, m.step);
+}
+
+// LVSA expanded window of frame t: W grows from {t}, right then left alternately (the other
+// side at a sequence end), until |G_s union W| = min(C, T).
+__device__ __forceinline__ void lvsa_window(const MaskDev& m, int64_t t, int64_t& lo, int64_t& hi) {
+  const int64_t T = m.frames;
+  const int64_t target = min(m.budget, T);
+  int64_t count = min(m.anchors, T) + (is_anchor_of(t, T, m.anchors, m.step) ? 0 : 1);
+  lo = hi = t;
+  bool right = true;
+  while (count < target) {
+    const bool can_r = hi + 1 < T, can_l = lo > 0;
+    if (!can_r && !can_l) break;
+    int64_t f;
+    if ((right && can_r) || !can_l) f = ++hi; else f = --lo;
+    if (!is_anchor_of(f, T, m.anchors, m.step)) ++count;
+    right = !right;
+  }
 }
 
 // Parametric predicate for rows of the non-static kinds.
@@ -57,6 +80,15 @@ __device__ __forceinline__ bool predicate(const MaskDev& m, int64_t i, int64_t j
       return true;
     case kTwoStage:
       return (j / m.group == i / m.group) || (j == (i + m.group) % m.nb);
+    case kLvsaFrames: {
+      // lo_i / hi_i hold the union of the windows of i's frames
+      int64_t lo_j, hi_j;
+      block_units(m, j, lo_j, hi_j);
+      if (lo_j <= hi_i && hi_j >= lo_i) return true;
+      for (int64_t f = lo_j; f <= hi_j; ++f)
+        if (is_anchor_of(f, m.frames, m.anchors, m.step)) return true;
+      return false;
+    }
     default: {
       int64_t lo_j, hi_j;
       block_units(m, j, lo_j, hi_j);
@@ -127,6 +159,19 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) mask_rows_kernel(MaskDev 
   } else {
     int64_t lo_i = 0, hi_i = 0;
     if (m.kind == kWindowAnchor) block_units(m, i, lo_i, hi_i);
+    if (m.kind == kLvsaFrames) {
+      // union of the (contiguous, overlapping) windows of the frames block i touches
+      int64_t f0, f1;
+      block_units(m, i, f0, f1);
+      lo_i = m.frames;
+      hi_i = -1;
+      for (int64_t t = f0; t <= f1; ++t) {
+        int64_t wl, wh;
+        lvsa_window(m, t, wl, wh);
+        lo_i = min(lo_i, wl);
+        hi_i = max(hi_i, wh);
+      }
+    }
     for (int64_t j0 = 0; j0 < m.nb; j0 += 32) {
       const int64_t j = j0 + lane;
       const bool set = predicate(m, i, j, lo_i, hi_i);
@@ -206,6 +251,8 @@ cudaError_t launch_build_mask(const MaskArgs& a, cudaStream_t stream) {
   m.anchors = a.num_anchors;
   m.step = a.step;
   m.group = a.group_blocks > 0 ? a.group_blocks : 1;
+  m.frames = (a.n_valid + m.unit - 1) / m.unit;
+  m.budget = a.budget_frames;
   m.dense = a.dense;
   const unsigned blocks = unsigned((m.rows + kWarpsPerBlock - 1) / kWarpsPerBlock);
   mask_rows_kernel<false><<<blocks, kWarpsPerBlock * 32, 0, stream>>>(m, a.row_ptr, a.col_idx);

@@ -27,6 +27,9 @@ def mask_params_for(spec: dict, n_pad: int, n_valid: int, block_size: int, mask_
         return lb.MaskParams(lb.LVA_MASK_TWO_STAGE, n_pad, n_valid, block_size, 1, group_blocks=spec["group"])
     if kind == "all":
         return lb.MaskParams(lb.LVA_MASK_ALL, n_pad, n_valid, block_size, 1)
+    if kind == "lvsa_frames":
+        return lb.MaskParams(lb.LVA_MASK_LVSA_FRAMES, n_pad, n_valid, block_size, 1, spec["unit"],
+                             num_anchors=spec["anchors"], step=step, budget_frames=spec["budget"])
     if kind == "static":
         return lb.MaskParams(lb.LVA_MASK_STATIC, n_pad, n_valid, block_size, mask_heads)
     raise ValueError(f"unknown mask kind {kind!r}")
@@ -77,7 +80,7 @@ class VideoBlockSparseAttention:
 
     def build_mask(self, step: int = 0):
         """(Re)build the CSR; parametric window masks depend on the denoising step."""
-        steps_matter = self.mask["kind"] == "window_anchor" and self.mask.get("anchors", 0) > 0
+        steps_matter = self.mask["kind"] in ("window_anchor", "lvsa_frames") and self.mask.get("anchors", 0) > 0
         key = step if steps_matter else 0
         if self._built_step == key:
             return

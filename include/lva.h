@@ -87,7 +87,8 @@ typedef enum {
   LVA_MASK_WINDOW_ANCHOR = 0,  /* local window + rotating global anchors (LVSA)      */
   LVA_MASK_STATIC = 1,         /* a given dense per-head block mask (CalibAtt-style) */
   LVA_MASK_ALL = 2,            /* every block: dense attention                       */
-  LVA_MASK_TWO_STAGE = 3       /* local window groups + one strided block (SQuad-style) */
+  LVA_MASK_TWO_STAGE = 3,      /* local window groups + one strided block (SQuad-style) */
+  LVA_MASK_LVSA_FRAMES = 4     /* expanded frame windows + rotating global frames (LVSA) */
 } lva_mask_kind;
 
 typedef struct {
@@ -101,6 +102,7 @@ typedef struct {
   int num_anchors;             /* WINDOW_ANCHOR: G >= 0 anchor key blocks */
   int step;                    /* WINDOW_ANCHOR: denoising step s >= 0 */
   int group_blocks;            /* TWO_STAGE: g >= 1 blocks per local window group */
+  int budget_frames;           /* LVSA_FRAMES: C >= 1 attended frames per query frame */
 } lva_mask_params;
 
 /* Upper bound on the CSR entries of a mask: mask_heads * nb * nb (0 on bad params). */
@@ -126,6 +128,15 @@ int64_t lva_block_mask_max_nnz(const lva_mask_params* params);
  *     Video Generation", technical summary section 1: local pass in windows of w tokens,
  *     global pass across windows at the same relative position):
  *     M[i][j] = (floor(j/g) == floor(i/g))  or  j == (i + g) mod nb.
+ *   LVSA_FRAMES (LVSA page, technical summary section 2, "Ancore Globali Rotanti" and
+ *     "Finestre Adattive Espanse": global frames rotate with the step; the local window is
+ *     extended where it overlaps global frames so that a query frame attends C frames).
+ *     Frames f = 0..T-1 of U = window_unit_tokens tokens, T = ceil(n_valid / U); global
+ *     frames G_s = { (floor(a*T/G) + s) mod T : a < G }.  W(t) starts as {t} and grows one
+ *     frame at a time, right then left alternately (the other side when one end is reached),
+ *     until |G_s union W(t)| = min(C, T); A(t) = G_s union W(t).  Query block i attends key
+ *     block j when a frame of j lies in A(t) for a frame t of i (frames of real tokens; a
+ *     padding-only block takes the last frame).
  *
  * Outputs (device): row_ptr [mask_heads*nb + 1] (row_ptr[0] = 0), col_idx [col_capacity],
  * *nnz_out = row_ptr[mask_heads*nb].  Columns of a row are ascending and unique.

@@ -28,6 +28,12 @@ Readings where the pages are silent (each listed in the design notes):
 * Two-stage: window groups of g consecutive blocks (the last group may be short).  Local
   pass: j in the same group as i.  Global pass: one strided block j = (i + g) mod nb,
   the same relative position in the next group.
+* Expanded adaptive windows with frame anchors (LVSA technical summary section 2, "Finestre
+  Adattive Espanse" and "Ancore Globali Rotanti"): frames t = 0..T-1 (U tokens each); the
+  global frames G_s = {(floor(a*T/G) + s) mod T}; the local window W(t) starts as {t} and
+  grows one frame at a time -- right, then left, alternately, continuing on the other side
+  at a sequence end -- until |G_s union W(t)| = min(C, T) for the budget C.  A query block
+  attends the union of A(t) over the frames its real tokens touch.
 """
 from __future__ import annotations
 
@@ -109,4 +115,59 @@ def csr_to_dense(row_ptr: np.ndarray, col_idx: np.ndarray, mask_heads: int, nb: 
     for r in range(mask_heads * nb):
         for c in col_idx[row_ptr[r]:row_ptr[r + 1]]:
             m[r // nb, r % nb, c] = True
+    return m
+
+
+def lvsa_frame_sets(num_frames: int, num_anchors: int, step: int, budget: int):
+    """A(t) = G_s union W(t) for every frame t, grown frame by frame as described above.
+
+    Returns (anchors, windows, sets): anchors as a set, windows[t] = (lo, hi), sets[t] = A(t).
+    """
+    T = num_frames
+    anchors = {(a * T // num_anchors + step) % T for a in range(num_anchors)} if num_anchors else set()
+    target = min(budget, T)
+    windows, sets = [], []
+    for t in range(T):
+        lo = hi = t
+        attended = anchors | {t}
+        turn_right = True
+        while len(attended) < target:
+            can_right, can_left = hi + 1 < T, lo - 1 >= 0
+            if not (can_right or can_left):
+                break
+            if (turn_right and can_right) or not can_left:
+                hi += 1
+                attended.add(hi)
+            else:
+                lo -= 1
+                attended.add(lo)
+            turn_right = not turn_right
+        windows.append((lo, hi))
+        sets.append(attended)
+    return anchors, windows, sets
+
+
+def lvsa_frame_mask(n_pad: int, n_valid: int, block_size: int, frame_tokens: int,
+                    num_anchors: int, step: int, budget: int) -> np.ndarray:
+    """Dense boolean [nb, nb] block mask of the expanded-window LVSA pattern."""
+    bs = block_size
+    nb = n_pad // bs
+    T = (n_valid + frame_tokens - 1) // frame_tokens
+    _, _, sets = lvsa_frame_sets(T, num_anchors, step, budget)
+
+    def frames_of(i):
+        first = i * bs
+        if first >= n_valid:
+            f = (n_valid - 1) // frame_tokens
+            return range(f, f + 1)
+        last = min((i + 1) * bs, n_valid) - 1
+        return range(first // frame_tokens, last // frame_tokens + 1)
+
+    m = np.zeros((nb, nb), dtype=bool)
+    for i in range(nb):
+        attended = set()
+        for t in frames_of(i):
+            attended |= sets[t]
+        for j in range(nb):
+            m[i, j] = any(f in attended for f in frames_of(j))
     return m

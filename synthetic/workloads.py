@@ -154,7 +154,8 @@ def mask_variants(w: Workload) -> List[dict]:
 
     ``window_anchor`` entries give (unit tokens, radius in units, anchors, steps);
     ``static`` entries carry a dense per-head mask; ``two_stage`` gives the window group
-    size in blocks; ``all`` is the dense mask.
+    size in blocks; ``all`` is the dense mask; ``lvsa_frames`` gives (frame tokens, global
+    frames, frame budget, steps).
     """
     if w.name == "tiny":
         return [dict(label="win1_anchor1", kind="window_anchor", unit=w.block_size, radius=1,
@@ -174,5 +175,9 @@ def mask_variants(w: Workload) -> List[dict]:
         return ([dict(label="two_stage", kind="two_stage", group=g)]
                 + [dict(label=f"band{r}_anchor4", kind="window_anchor", unit=w.block_size,
                         radius=r, anchors=4, steps=[0]) for r in (23, 48, 130, 287)]
-                + [dict(label="all", kind="all")])
+                + [dict(label="all", kind="all")]
+                # expanded frame windows: a 21-frame budget (a Wan-2.1-like training horizon)
+                # with 4 rotating global frames over the 81 latent frames
+                + [dict(label="lvsa_c21_g4", kind="lvsa_frames", unit=w.frame_tokens, anchors=4,
+                        budget=21, steps=[0])])
     raise KeyError(w.name)

@@ -12,7 +12,7 @@ import pytest
 import torch
 
 from oracle.attention import attention_blocked
-from oracle.mask import all_mask, dense_to_csr, two_stage_mask, window_anchor_mask
+from oracle.mask import all_mask, dense_to_csr, lvsa_frame_mask, two_stage_mask, window_anchor_mask
 from oracle.reorder import reorder_forward, tile_permutation
 from synthetic import WORKLOADS, make_qkv, mask_variants, static_calibrated_mask
 from tests.gpu_helpers import check_o_lse, require_gpu
@@ -135,6 +135,9 @@ def _oracle_mask(w, spec, step):
         return two_stage_mask(w.nb, spec["group"])[None]
     if spec["kind"] == "all":
         return all_mask(w.nb)[None]
+    if spec["kind"] == "lvsa_frames":
+        return lvsa_frame_mask(w.n_pad, w.n_valid, w.block_size, spec["unit"], spec["anchors"], step,
+                               spec["budget"])[None]
     return static_calibrated_mask(w).astype(bool)
 
 
@@ -210,4 +213,4 @@ def test_workload_large():
 
 
 def test_workload_long():
-    _run_workload("long", {"two_stage", "band23_anchor4", "all"}, per_head=1)
+    _run_workload("long", {"two_stage", "band23_anchor4", "all", "lvsa_c21_g4"}, per_head=1)

@@ -81,6 +81,12 @@ def test_sweeps(name):
             p = lva.MaskParams(lva.LVA_MASK_TWO_STAGE, w.n_pad, w.n_valid, w.block_size, 1,
                                group_blocks=spec["group"])
             ref = two_stage_mask(w.nb, spec["group"])
+        elif spec["kind"] == "lvsa_frames":
+            from oracle.mask import lvsa_frame_mask
+            p = lva.MaskParams(lva.LVA_MASK_LVSA_FRAMES, w.n_pad, w.n_valid, w.block_size, 1, spec["unit"],
+                               num_anchors=spec["anchors"], step=0, budget_frames=spec["budget"])
+            ref = lvsa_frame_mask(w.n_pad, w.n_valid, w.block_size, spec["unit"], spec["anchors"], 0,
+                                  spec["budget"])
         else:
             p = lva.MaskParams(lva.LVA_MASK_ALL, w.n_pad, w.n_valid, w.block_size)
             ref = all_mask(w.nb)
@@ -110,3 +116,20 @@ def test_edge_cases():
     for nb, g in [(10, 3), (7, 7), (5, 1), (9, 20)]:
         p = lva.MaskParams(lva.LVA_MASK_TWO_STAGE, nb * 128, nb * 128, 128, 1, group_blocks=g)
         _check(p, two_stage_mask(nb, g))
+
+
+@pytest.mark.parametrize("n_pad,n_valid,bs,U,G,C,steps", [
+    (32768, 32760, 128, 1560, 4, 8, (0, 3, 11)),       # small workload grid, 21 frames
+    (126464, 126360, 128, 1560, 4, 21, (0, 5)),        # long workload grid, 81 frames, budget 21
+    (256, 256, 64, 64, 1, 2, (0, 1, 2, 3)),            # tiny: one block per frame
+    (6400, 6375, 128, 100, 5, 17, (0, 9)),             # frames of 100 tokens: blocks span 2-3 frames
+    (4096, 4000, 128, 1000, 2, 9, (1,)),               # budget above the frame count (4 frames)
+    (8192, 8192, 64, 512, 0, 5, (0,)),                 # no global frames: symmetric windows
+])
+def test_lvsa_frames(n_pad, n_valid, bs, U, G, C, steps):
+    import block_sparse_attention_lva_b200 as lva
+    from oracle.mask import lvsa_frame_mask
+    for s in steps:
+        p = lva.MaskParams(lva.LVA_MASK_LVSA_FRAMES, n_pad, n_valid, bs, 1, U, num_anchors=G, step=s,
+                           budget_frames=C)
+        _check(p, lvsa_frame_mask(n_pad, n_valid, bs, U, G, s, C))

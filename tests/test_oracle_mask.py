@@ -139,3 +139,56 @@ def test_csr_roundtrip_and_order():
         seg = ci[rp[row]:rp[row + 1]]
         assert np.all(np.diff(seg) > 0)
     assert np.array_equal(csr_to_dense(rp, ci, 3, 9), m)
+
+
+# ---------------------------------------------------------------- expanded LVSA windows
+from oracle.mask import lvsa_frame_mask, lvsa_frame_sets  # noqa: E402
+
+
+def test_lvsa_hand_worked_windows():
+    g = json.load(open(os.path.join(GOLDEN, "lvsa_frames_hand.json")))
+    for c in g["cases"]:
+        anchors, windows, sets = lvsa_frame_sets(c["T"], c["G"], c["step"], c["C"])
+        assert sorted(anchors) == c["anchors"]
+        assert [list(w) for w in windows] == c["windows"], c["why"]
+
+
+@pytest.mark.parametrize("T,G,C", [(21, 4, 21), (81, 4, 21), (126, 6, 21), (10, 3, 4), (5, 2, 9), (30, 0, 7)])
+def test_lvsa_budget_invariant(T, G, C):
+    # LVSA: the window is extended where it overlaps global frames so that |A(t)| = C
+    # (or every frame when C >= T), at every step; W(t) is a contiguous interval holding t.
+    for s in (0, 1, 7):
+        anchors, windows, sets = lvsa_frame_sets(T, G, s, C)
+        assert len(anchors) == min(G, T)
+        for t, (lo, hi) in enumerate(windows):
+            assert lo <= t <= hi
+            assert sets[t] == anchors | set(range(lo, hi + 1))
+            assert len(sets[t]) == min(C, T)
+
+
+def test_lvsa_without_anchors_is_the_symmetric_window_inside():
+    # G = 0, C = 2r + 1: interior frames get exactly [t - r, t + r].
+    T, r = 40, 3
+    _, windows, _ = lvsa_frame_sets(T, 0, 0, 2 * r + 1)
+    for t in range(r, T - r):
+        assert windows[t] == (t - r, t + r)
+    assert windows[0] == (0, 2 * r) and windows[T - 1] == (T - 1 - 2 * r, T - 1)   # shifted inward
+
+
+def test_lvsa_pairs_linear_in_frames():
+    # Fixed budget: frame pairs = T * min(C, T), linear in T (LVSA complexity statement).
+    for T in (30, 60, 120):
+        _, _, sets = lvsa_frame_sets(T, 4, 0, 21)
+        assert sum(len(a) for a in sets) == 21 * T
+
+
+def test_lvsa_block_mask_from_frames():
+    # Blocks aligned to frames (2 blocks per frame): block-level mask = frame-level sets expanded.
+    T, fb, bs = 12, 2, 64
+    U = fb * bs
+    n = T * U
+    m = lvsa_frame_mask(n, n, bs, U, 3, 2, 5)
+    _, _, sets = lvsa_frame_sets(T, 3, 2, 5)
+    for i in range(T * fb):
+        for j in range(T * fb):
+            assert m[i, j] == ((j // fb) in sets[i // fb])
