@@ -46,7 +46,8 @@ SIGNATURES = {
     "lva_block_mask_max_nnz": (_c_i64, [ctypes.POINTER(LvaMaskParams)]),
     "lva_build_block_mask": (_c_int, [ctypes.POINTER(LvaMaskParams), _vp, _vp, _vp, _c_i64, _vp, _vp]),
     "lva_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
-                                       _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp]),
+                                       _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp, _c_int, _vp]),
+    "lva_broadcast_blocks": (_c_int, [_vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _vp, _c_int, _vp]),
     "lva_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
 }
 
@@ -168,9 +169,17 @@ def lva_build_block_mask(params: MaskParams, dense_mask, row_ptr, col_idx, nnz_o
     return row_ptr, col_idx, nnz_out
 
 
+def _check_query_src(query_src, H, nb):
+    import torch
+    _cuda_tensor(query_src, "query_src", torch.int32)
+    _need(query_src.dim() == 2 and query_src.shape[0] in (1, H) and query_src.shape[1] == nb,
+          f"query_src must have shape [1 or {H}, {nb}]")
+
+
 def lva_block_sparse_attn(q, k, v, o, lse, n_valid: int, block_size: int, row_ptr, col_idx,
-                          mask_heads: int, scale: float):
-    """O, LSE of block-sparse softmax attention over the CSR-listed key blocks."""
+                          mask_heads: int, scale: float, query_src=None):
+    """O, LSE of block-sparse softmax attention over the CSR-listed key blocks.  With
+    ``query_src`` ([1 or H, nb] int32), blocks whose source is another block are skipped."""
     import torch
     B, H, n_pad, d = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
@@ -180,10 +189,26 @@ def lva_block_sparse_attn(q, k, v, o, lse, n_valid: int, block_size: int, row_pt
     nb = n_pad // block_size
     _cuda_tensor(row_ptr, "row_ptr", torch.int32, mask_heads * nb + 1)
     _cuda_tensor(col_idx, "col_idx", torch.int32)
+    src_heads = 1
+    if query_src is not None:
+        _check_query_src(query_src, H, nb)
+        src_heads = query_src.shape[0]
     _check(lib.lva_block_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, n_pad, n_valid,
                                      d, block_size, _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
-                                     mask_heads, ctypes.c_float(scale),
+                                     mask_heads, ctypes.c_float(scale), _ptr(query_src), src_heads,
                                      ctypes.c_void_p(_stream(q.device))))
+    return o, lse
+
+
+def lva_broadcast_blocks(o, lse, block_size: int, query_src):
+    """Copy O rows and LSE of anchor blocks into the blocks that name them in ``query_src``."""
+    import torch
+    B, H, n_pad, d = o.shape
+    _cuda_tensor(o, "o", torch.bfloat16)
+    _cuda_tensor(lse, "lse", torch.float32, B * H * n_pad)
+    _check_query_src(query_src, H, n_pad // block_size)
+    _check(lib.lva_broadcast_blocks(_ptr(o), _ptr(lse), B, H, n_pad, d, block_size, _ptr(query_src),
+                                    query_src.shape[0], ctypes.c_void_p(_stream(o.device))))
     return o, lse
 
 

@@ -178,7 +178,8 @@ lva_status lva_build_block_mask(const lva_mask_params* p, const uint8_t* dense_m
 lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, void* o, float* lse,
                                  int B, int H, int64_t n_pad, int64_t n_valid, int d, int block_size,
                                  const int32_t* row_ptr, const int32_t* col_idx, int64_t col_len,
-                                 int mask_heads, float scale, cudaStream_t stream) {
+                                 int mask_heads, float scale, const int32_t* query_src, int src_heads,
+                                 cudaStream_t stream) {
   if (B < 0 || H < 1) return fail(LVA_ERR_INVALID_ARG, "attn: need B >= 0 and H >= 1");
   if (d != 64 && d != 128) return fail(LVA_ERR_UNSUPPORTED, "attn: head dim must be 64 or 128");
   if (block_size != 64 && block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "attn: block_size must be 64 or 128");
@@ -188,6 +189,10 @@ lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, vo
   if (int64_t(B) * H * n_pad >= (int64_t(1) << 31)) return fail(LVA_ERR_UNSUPPORTED, "attn: B*H*n_pad must be < 2^31");
   if (!(scale == scale)) return fail(LVA_ERR_INVALID_ARG, "attn: scale is NaN");
   if (col_len < 0) return fail(LVA_ERR_INVALID_ARG, "attn: col_len < 0");
+  if (query_src != nullptr && src_heads != 1 && src_heads != H)
+    return fail(LVA_ERR_INVALID_ARG, "attn: src_heads must be 1 or H");
+  if (query_src != nullptr && !aligned(query_src, 4))
+    return fail(LVA_ERR_INVALID_ARG, "attn: query_src must be 4-byte aligned");
   if (B == 0) return ok();
   if (!q || !k || !v || !o || !lse || !row_ptr || (!col_idx && col_len > 0))
     return fail(LVA_ERR_INVALID_ARG, "attn: null pointer");
@@ -198,11 +203,29 @@ lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, vo
   int* err = device_error_word();
   if (err == nullptr) return fail(LVA_ERR_CUDA, "attn: cannot locate the device error word");
   AttnArgs a{q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr,
-             col_idx, col_len, mask_heads, scale, err};
+             col_idx, col_len, mask_heads, scale, query_src, src_heads, err};
   const char* why = "launch";
   cudaError_t e = launch_attn(a, stream, &why);
   if (e != cudaSuccess) return fail(LVA_ERR_CUDA, "attn: %s: %s", why, cudaGetErrorString(e));
   return ok();
+}
+
+lva_status lva_broadcast_blocks(void* o, float* lse, int B, int H, int64_t n_pad, int d, int block_size,
+                                const int32_t* query_src, int src_heads, cudaStream_t stream) {
+  if (B < 0 || H < 1) return fail(LVA_ERR_INVALID_ARG, "broadcast: need B >= 0 and H >= 1");
+  if (d != 64 && d != 128) return fail(LVA_ERR_UNSUPPORTED, "broadcast: head dim must be 64 or 128");
+  if (block_size != 64 && block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "broadcast: block_size must be 64 or 128");
+  if (n_pad <= 0 || n_pad % block_size != 0) return fail(LVA_ERR_INVALID_ARG, "broadcast: n_pad must be a positive multiple of block_size");
+  if (src_heads != 1 && src_heads != H) return fail(LVA_ERR_INVALID_ARG, "broadcast: src_heads must be 1 or H");
+  if (int64_t(B) * H * n_pad >= (int64_t(1) << 31)) return fail(LVA_ERR_UNSUPPORTED, "broadcast: B*H*n_pad must be < 2^31");
+  if (B == 0) return ok();
+  if (!o || !lse || !query_src) return fail(LVA_ERR_INVALID_ARG, "broadcast: null pointer");
+  if (!aligned(o, 16) || !aligned(lse, 4) || !aligned(query_src, 4))
+    return fail(LVA_ERR_INVALID_ARG, "broadcast: o must be 16-byte, lse and query_src 4-byte aligned");
+  int* err = device_error_word();
+  if (err == nullptr) return fail(LVA_ERR_CUDA, "broadcast: cannot locate the device error word");
+  BroadcastArgs a{o, lse, B, H, n_pad, d, block_size, query_src, src_heads, err};
+  return from_cuda(launch_broadcast(a, stream), "broadcast launch");
 }
 
 lva_status lva_device_error(cudaStream_t stream, lva_status* status, int* detail) {

@@ -67,6 +67,8 @@ struct AttnParams {
   int64_t col_len;
   __nv_bfloat16* o;
   float* lse;
+  const int32_t* query_src;        // NULL or [src_heads, nb]: blocks copied from an anchor
+  int src_heads;
   int* err;
 };
 
@@ -153,6 +155,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   const int64_t plane = item / p.nb;
   const int i = int(item - plane * p.nb);
   const int h = int(plane % p.H);
+  // Blocks of repetitive heads that take an anchor's output are not computed here.
+  if (p.query_src != nullptr &&
+      __ldg(p.query_src + int64_t(p.src_heads == 1 ? 0 : h) * p.nb + i) != i)
+    return;
   const int64_t csr = int64_t(p.mask_heads == 1 ? 0 : h) * p.nb + i;
   int32_t start;
   bool bad;
@@ -530,6 +536,8 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   p.col_len = a.col_len;
   p.o = static_cast<__nv_bfloat16*>(a.o);
   p.lse = a.lse;
+  p.query_src = a.query_src;
+  p.src_heads = a.src_heads;
   p.err = a.err;
   const int64_t items = rows / a.block_size;
   if (items == 0) return cudaSuccess;

@@ -47,9 +47,23 @@ struct AttnArgs {
   int64_t col_len;
   int mask_heads;
   float scale;
+  const int32_t* query_src;  // NULL or [src_heads, nb]
+  int src_heads;
   int* err;  // device error word
 };
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why);
+
+struct BroadcastArgs {
+  void* o;
+  float* lse;
+  int B, H;
+  int64_t n_pad;
+  int d, block_size;
+  const int32_t* query_src;
+  int src_heads;
+  int* err;
+};
+cudaError_t launch_broadcast(const BroadcastArgs& a, cudaStream_t stream);
 
 // Device error word of the current device (from api.cu).
 int* device_error_word();

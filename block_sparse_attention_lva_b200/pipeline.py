@@ -39,11 +39,13 @@ class VideoBlockSparseAttention:
     """Block-sparse self-attention over a T x Hg x Wg latent video grid.
 
     ``mask`` is a specification dict; for ``kind == "static"`` pass the dense per-head block
-    mask (uint8 [H_m, nb, nb], any device) as ``static_mask``.
+    mask (uint8 [H_m, nb, nb], any device) as ``static_mask``.  ``query_src`` ([1 or H, nb]
+    int32) marks repetitive heads: their non-anchor query blocks are not computed and take
+    the output of the anchor block they name.
     """
 
     def __init__(self, B, H, d, grid, tile, block_size, mask: dict, static_mask=None,
-                 scale=None, device="cuda"):
+                 scale=None, device="cuda", query_src=None):
         self.B, self.H, self.d = B, H, d
         self.grid, self.tile, self.block_size = tuple(grid), tuple(tile), block_size
         self.n_valid = grid[0] * grid[1] * grid[2]
@@ -76,6 +78,8 @@ class VideoBlockSparseAttention:
         self.row_ptr = torch.empty(self.mask_heads * self.nb + 1, dtype=torch.int32, **kw)
         self.col_idx = torch.empty(cap, dtype=torch.int32, **kw)
         self.nnz = torch.empty(1, dtype=torch.int32, **kw)
+        self.query_src = (torch.as_tensor(query_src, dtype=torch.int32).to(self.device).contiguous()
+                          if query_src is not None else None)
         self._built_step = None
 
     def build_mask(self, step: int = 0):
@@ -111,7 +115,10 @@ class VideoBlockSparseAttention:
 
     def attend(self):
         lb.lva_block_sparse_attn(self.q_t, self.k_t, self.v_t, self.o_t, self.lse, self.n_valid,
-                                 self.block_size, self.row_ptr, self.col_idx, self.mask_heads, self.scale)
+                                 self.block_size, self.row_ptr, self.col_idx, self.mask_heads, self.scale,
+                                 self.query_src)
+        if self.query_src is not None:
+            lb.lva_broadcast_blocks(self.o_t, self.lse, self.block_size, self.query_src)
 
     def reorder_out(self):
         P = self.B * self.H

@@ -168,6 +168,9 @@ lva_status lva_build_block_mask(const lva_mask_params* params, const uint8_t* de
  * row_ptr: device [mask_heads*nb + 1]; col_idx: device, col_len entries (the kernel never
  * reads past col_len; CSR entries out of range are skipped and reported through
  * lva_device_error as LVA_ERR_INVALID_ARG).
+ * query_src: NULL, or device int32 [src_heads, nb] (src_heads in {1, H}): query blocks with
+ * query_src[h_s*nb + i] != i are not computed here (their O/LSE are left untouched for
+ * lva_broadcast_blocks to fill).
  * Supported: d in {64, 128}, block_size in {64, 128}, mask_heads in {1, H},
  * B*H*n_pad < 2^31.
  */
@@ -175,7 +178,26 @@ lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, vo
                                  int B, int H, int64_t n_pad, int64_t n_valid, int d,
                                  int block_size, const int32_t* row_ptr, const int32_t* col_idx,
                                  int64_t col_len, int mask_heads, float scale,
-                                 cudaStream_t stream);
+                                 const int32_t* query_src, int src_heads, cudaStream_t stream);
+
+/*
+ * lva_broadcast_blocks -- fill the query blocks of repetitive heads from their anchors.
+ *
+ * CalibAtt page ("Accelerating Text-to-Video Generation with Calibrated Sparse Attention",
+ * section 2 A.3 and B): for a head whose spatial rows repeat, attention is computed only for
+ * anchor rows and the result is replicated to the other rows.  At block granularity in tile
+ * order: query_src[h_s*nb + i] (h_s = (src_heads == 1 ? 0 : h)) names the block whose output
+ * block i takes; query_src[h_s*nb + i] == i marks a computed (anchor) block.  Run after
+ * lva_block_sparse_attn with the same query_src (which skips the non-anchor blocks):
+ *   O[b][h][i*Bs + r][:] = O[b][h][src*Bs + r][:],  LSE[b][h][i*Bs + r] = LSE[b][h][src*Bs + r]
+ * for every block i with src = query_src[...] != i and r < Bs.
+ * o: device bf16 [B, H, n_pad, d], 16-byte aligned; lse: device fp32 [B, H, n_pad].
+ * A source outside [0, nb) or one that is not itself an anchor is skipped and reported
+ * through lva_device_error as LVA_ERR_INVALID_ARG (detail = the offending map entry index).
+ */
+lva_status lva_broadcast_blocks(void* o, float* lse, int B, int H, int64_t n_pad, int d,
+                                int block_size, const int32_t* query_src, int src_heads,
+                                cudaStream_t stream);
 
 /*
  * lva_device_error -- read and clear the current device's kernel error word.

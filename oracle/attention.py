@@ -113,3 +113,34 @@ def attention_bruteforce(q, k, v, masks, block_size: int, n_valid: int, scale: f
                 out[b, h, r] = (w / w.sum()) @ v[b, h]
                 lse[b, h, r] = mx + np.log(w.sum())
     return out, lse
+
+
+def attention_with_broadcast(q, k, v, masks, block_size: int, n_valid: int, scale: float, query_src):
+    """Repetitive heads: only anchor query blocks are computed, the others copy an anchor.
+
+    CalibAtt page ("Accelerating Text-to-Video Generation with Calibrated Sparse Attention"),
+    section 2 A.3 and B: for a head marked repetitive, attention is computed for a subset of
+    rows (the anchors) and the result is replicated to the other rows.  Reading (block
+    granularity, tile order): ``query_src`` [S, nb] (S in {1, H}) names for every query block
+    i the block whose O rows and LSE it takes; query_src[h][i] == i marks a computed block,
+    and every source must itself be computed.
+    """
+    q_, k_, v_ = _as_f64(q), _as_f64(k), _as_f64(v)
+    src = np.asarray(query_src)
+    if src.ndim == 1:
+        src = src[None]
+    B, H, n_pad, d = q_.shape
+    nb = n_pad // block_size
+    blocks = [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)
+              if src[h if src.shape[0] == H else 0, i] == i]
+    out, lse = attention_blocked(q, k, v, masks, block_size, n_valid, scale, query_blocks=blocks)
+    for b in range(B):
+        for h in range(H):
+            row = src[h if src.shape[0] == H else 0]
+            for i in range(nb):
+                j = int(row[i])
+                if j != i:
+                    assert row[j] == j, "a source block must be computed"
+                    out[b, h, i * block_size:(i + 1) * block_size] = out[b, h, j * block_size:(j + 1) * block_size]
+                    lse[b, h, i * block_size:(i + 1) * block_size] = lse[b, h, j * block_size:(j + 1) * block_size]
+    return out, lse

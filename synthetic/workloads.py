@@ -181,3 +181,45 @@ def mask_variants(w: Workload) -> List[dict]:
                 + [dict(label="lvsa_c21_g4", kind="lvsa_frames", unit=w.frame_tokens, anchors=4,
                         budget=21, steps=[0])])
     raise KeyError(w.name)
+
+
+def spatial_repetition_map(w: Workload, repetitive_heads, group_tile_rows: int) -> np.ndarray:
+    """Block source map [H, nb] (int32) for heads whose spatial rows repeat.
+
+    An input, like a calibrated mask: CalibAtt selects repetitive heads offline from the
+    similarity of spatial rows, which needs model activations.  Here, in tile order with
+    tiles of (1, th, tw) tokens, the tiles of a frame form a grid of tile rows x tile
+    columns; for the listed heads every group of ``group_tile_rows`` consecutive tile rows
+    takes the output of its first tile row (the anchor), column by column.  A block is
+    repeated only when it is one full tile and its anchor tile is full too; every other
+    block is computed.  Other heads compute every block.
+    """
+    tt, th, tw = w.tile
+    assert tt == 1 and th * tw == w.block_size
+    n_th = (w.Hg + th - 1) // th
+    n_tw = (w.Wg + tw - 1) // tw
+    # tile sizes and tile-order offsets inside one frame
+    offs, sizes = [], []
+    pos = 0
+    for ih in range(n_th):
+        for iw in range(n_tw):
+            size = min(th, w.Hg - ih * th) * min(tw, w.Wg - iw * tw)
+            offs.append(pos)
+            sizes.append(size)
+            pos += size
+    src = np.tile(np.arange(w.nb, dtype=np.int32), (w.H, 1))
+    for t in range(w.T):
+        base = t * w.frame_tokens
+        for ih in range(n_th):
+            a_ih = ih - ih % group_tile_rows
+            if a_ih == ih:
+                continue
+            for iw in range(n_tw):
+                me, an = ih * n_tw + iw, a_ih * n_tw + iw
+                start, a_start = base + offs[me], base + offs[an]
+                if (sizes[me] != w.block_size or sizes[an] != w.block_size
+                        or start % w.block_size or a_start % w.block_size):
+                    continue
+                for h in repetitive_heads:
+                    src[h, start // w.block_size] = a_start // w.block_size
+    return src

@@ -58,7 +58,7 @@ def test_attn_argument_checks_fail_before_launch():
     call = lambda **kw: lib.lva_block_sparse_attn(
         kw.get("q", vp), vp, vp, vp, vp, kw.get("B", 1), kw.get("H", 2), kw.get("n_pad", 256),
         kw.get("n_valid", 256), kw.get("d", 128), kw.get("bs", 128), vp, vp, 10, kw.get("mh", 1),
-        ctypes.c_float(0.1), None)
+        ctypes.c_float(0.1), kw.get("qs", None), kw.get("sh", 1), None)
     assert call(d=96) == 2                       # unsupported head dim
     assert call(bs=32) == 2                      # unsupported block size
     assert call(n_pad=200) == 1                  # not a multiple of the block
@@ -67,6 +67,11 @@ def test_attn_argument_checks_fail_before_launch():
     assert call(q=ctypes.c_void_p(18)) == 1      # misaligned pointer
     assert b"aligned" in lib.lva_last_error_message()
     assert call(q=None) == 1
+    assert call(qs=vp, sh=3) == 1                # src_heads must be 1 or H
+    f = lib.lva_broadcast_blocks
+    assert f(vp, vp, 1, 2, 256, 96, 128, vp, 1, None) == 2     # head dim
+    assert f(vp, vp, 1, 2, 256, 128, 128, None, 1, None) == 1  # null map
+    assert f(vp, vp, 1, 2, 200, 128, 128, vp, 1, None) == 1    # n_pad
 
 
 def test_reorder_argument_checks_fail_before_launch():

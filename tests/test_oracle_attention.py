@@ -160,3 +160,37 @@ def test_padded_keys_never_matter():
     v2[:, :, n_valid:] = -7.0
     o2, l2 = attention_blocked(q, k2, v2, m, bs, n_valid, 0.25)
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_broadcast_identity_map_is_plain_attention():
+    from oracle.attention import attention_with_broadcast
+    n_pad, bs, d = 256, 64, 16
+    q, k, v = _inputs(1, 2, n_pad, d, 81)
+    m = np.random.default_rng(2).random((2, 4, 4)) < 0.6
+    ident = np.tile(np.arange(4, dtype=np.int32), (2, 1))
+    o1, l1 = attention_with_broadcast(q, k, v, m, bs, n_pad, 0.25, ident)
+    o2, l2 = attention_blocked(q, k, v, m, bs, n_pad, 0.25)
+    assert np.array_equal(np.nan_to_num(o1), np.nan_to_num(o2)) and np.array_equal(l1, l2)
+
+
+def test_broadcast_is_exact_when_rows_truly_repeat():
+    # CalibAtt: replicating anchor rows is exact when the repeated rows really repeat.  Give
+    # block 3 the queries and the key list of block 1: its output must equal the full result.
+    from oracle.attention import attention_with_broadcast
+    n_pad, bs, d = 256, 64, 16
+    q, k, v = _inputs(1, 1, n_pad, d, 91)
+    q[:, :, 3 * bs:4 * bs] = q[:, :, 1 * bs:2 * bs]
+    m = np.random.default_rng(3).random((1, 4, 4)) < 0.7
+    m[0, 1, 1] = True
+    m[0, 3] = m[0, 1]
+    src = np.array([[0, 1, 2, 1]], dtype=np.int32)
+    o1, l1 = attention_with_broadcast(q, k, v, m, bs, n_pad, 0.25, src)
+    o2, l2 = attention_blocked(q, k, v, m, bs, n_pad, 0.25)
+    assert np.max(np.abs(o1 - o2)) < 1e-12 and np.max(np.abs(l1 - l2)) < 1e-12
+
+
+def test_broadcast_source_must_be_an_anchor():
+    from oracle.attention import attention_with_broadcast
+    q, k, v = _inputs(1, 1, 192, 8, 5)
+    with pytest.raises(AssertionError):
+        attention_with_broadcast(q, k, v, np.ones((1, 3, 3), bool), 64, 192, 0.3, np.array([[1, 2, 2]]))
