@@ -381,7 +381,7 @@ def run_report(args):
     burst, sustained, hbm, peak_kind = _peaks()
     names = args.report.split(",")
     for name in names:
-        if name == "stress":
+        if name in ("stress", "squad"):
             continue
         w = WORKLOADS[name]
         q, k, v = make_qkv(w)
@@ -432,6 +432,24 @@ def run_report(args):
                                          "intercept_share_of_10pct": float(a / y[i10])}}), flush=True)
         del qd, kd, vd
         torch.cuda.empty_cache()
+    # SQuad's exact two-stage operator: 12 heads, 131,072 tokens (64 frames of 32 x 64),
+    # windows of 512 tokens (m = 256 windows): local pass, window transpose, global pass.
+    if "squad" in names:
+        H, n, d, win = 12, 131072, 128, 512
+        g = torch.Generator(device=dev).manual_seed(9)
+        qkv = torch.randn((3, 1, H, n, d), generator=g, device=dev).to(torch.bfloat16)
+        op = lva.SquadTwoPass(1, H, n, d, win, device=dev)
+        ms = _time_cuda(lambda: op(qkv[0], qkv[1], qkv[2]))
+        nbk = n // 128
+        pairs = H * nbk * (win // 128 + (n // win) // 128)
+        flops = pairs * 4.0 * 128 * 128 * d
+        print(json.dumps({"report": "squad_two_pass", "heads": H, "tokens": n, "window": win,
+                          "active_pairs": pairs, "ms": ms, "tflops": flops / ms / 1e9,
+                          "frac_of_burst": flops / ms / 1e9 / burst,
+                          "note": "2 attention launches + 3 transposes + inverse; FLOPs of both passes"}),
+              flush=True)
+        del qkv, op
+        torch.cuda.empty_cache()
     # mask-builder stress size: static mask, 40 heads x 4096 x 4096 blocks (671 MB read)
     if "stress" in names or args.report_stress:
         hm, nb = 40, 4096
@@ -457,7 +475,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--report", default="", help="comma list of workloads (tiny,small,static,large,long,stress): "
+    ap.add_argument("--report", default="", help="comma list of workloads (tiny,small,static,large,long,stress,squad): "
                     "per-mask kernel timings and the density sweep fit instead of the bench line")
     ap.add_argument("--report-stress", action="store_true")
     args = ap.parse_args()

@@ -144,3 +144,37 @@ def attention_with_broadcast(q, k, v, masks, block_size: int, n_valid: int, scal
                     out[b, h, i * block_size:(i + 1) * block_size] = out[b, h, j * block_size:(j + 1) * block_size]
                     lse[b, h, i * block_size:(i + 1) * block_size] = lse[b, h, j * block_size:(j + 1) * block_size]
     return out, lse
+
+
+def squad_two_pass(q, k, v, window: int, scale: float):
+    """SQuad's two-stage operator, token by token, in float64.
+
+    SQuad page ("SQuad: Sub-Quadratic Attention Distillation for Efficient Video
+    Generation"), technical summary section 1: a local pass mixes tokens inside fixed windows
+    of w tokens; a global pass mixes the tokens at the same relative position in every
+    window; the local output is the value stream of the global pass.  Reading: both passes
+    use the same Q and K; token k = a*w + p sits at position p of window a (n = m*w tokens).
+
+      O_L[a*w + p] = softmax_{p'} (scale q_{a*w+p} . k_{a*w+p'}) v_{a*w+p'}
+      O[a*w + p]   = softmax_{a'} (scale q_{a*w+p} . k_{a'*w+p}) O_L[a'*w+p]
+    """
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, H, n, d = q.shape
+    assert n % window == 0
+    m = n // window
+    sc = float(np.float32(scale))
+    o_local = np.empty_like(v)
+    out = np.empty_like(v)
+    for b in range(B):
+        for h in range(H):
+            for a in range(m):
+                idx = np.arange(a * window, (a + 1) * window)
+                s = sc * (q[b, h, idx] @ k[b, h, idx].T)
+                e = np.exp(s - s.max(axis=1, keepdims=True))
+                o_local[b, h, idx] = (e / e.sum(axis=1, keepdims=True)) @ v[b, h, idx]
+            for p in range(window):
+                idx = np.arange(p, n, window)
+                s = sc * (q[b, h, idx] @ k[b, h, idx].T)
+                e = np.exp(s - s.max(axis=1, keepdims=True))
+                out[b, h, idx] = (e / e.sum(axis=1, keepdims=True)) @ o_local[b, h, idx]
+    return out, o_local

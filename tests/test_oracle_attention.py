@@ -194,3 +194,53 @@ def test_broadcast_source_must_be_an_anchor():
     q, k, v = _inputs(1, 1, 192, 8, 5)
     with pytest.raises(AssertionError):
         attention_with_broadcast(q, k, v, np.ones((1, 3, 3), bool), 64, 192, 0.3, np.array([[1, 2, 2]]))
+
+
+# ---------------------------------------------------------------- SQuad two-stage operator
+def _sdpa64(q, k, v, scale, mask=None):
+    return torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double(),
+                                                            attn_mask=mask, scale=scale).numpy()
+
+
+def test_squad_one_window_is_dense_attention():
+    # w = n: one window, and every global group is a single token (attends itself).
+    from oracle.attention import squad_two_pass
+    q, k, v = _inputs(1, 2, 64, 16, 101)
+    o, _ = squad_two_pass(q, k, v, 64, 0.25)
+    assert np.max(np.abs(o - _sdpa64(q, k, v, 0.25))) < 1e-12
+
+
+def test_squad_unit_windows_is_dense_attention():
+    # w = 1: the local pass returns V, the global pass is dense attention over all tokens.
+    from oracle.attention import squad_two_pass
+    q, k, v = _inputs(1, 2, 48, 8, 103)
+    o, o_local = squad_two_pass(q, k, v, 1, 0.3)
+    assert np.max(np.abs(o_local - v.double().numpy())) < 1e-15
+    assert np.max(np.abs(o - _sdpa64(q, k, v, float(np.float32(0.3))))) < 1e-12
+
+
+def test_squad_matches_explicit_masked_matrices():
+    # Twin: the two passes as dense masked attention (library SDPA with boolean masks).
+    from oracle.attention import squad_two_pass
+    n, w = 96, 8
+    q, k, v = _inputs(1, 1, n, 16, 107)
+    idx = torch.arange(n)
+    local = (idx[:, None] // w) == (idx[None, :] // w)
+    glob = (idx[:, None] % w) == (idx[None, :] % w)
+    o_l = _sdpa64(q, k, v, 0.25, local)
+    o_ref = _sdpa64(q, k, torch.from_numpy(o_l), 0.25, glob)
+    o, o_local = squad_two_pass(q, k, v, w, 0.25)
+    assert np.max(np.abs(o_local - o_l)) < 1e-12 and np.max(np.abs(o - o_ref)) < 1e-12
+
+
+def test_squad_full_receptive_field():
+    # Composition recovers a full receptive field: every output depends on every value row.
+    from oracle.attention import squad_two_pass
+    n, w = 36, 6
+    q, k, v = _inputs(1, 1, n, 8, 109)
+    base, _ = squad_two_pass(q, k, v, w, 0.5)
+    for c in (0, 17, 35):
+        v2 = v.double().clone()
+        v2[0, 0, c] += 1.0
+        o2, _ = squad_two_pass(q, k, v2, w, 0.5)
+        assert np.all(np.abs(o2 - base).max(axis=-1) > 0)
