@@ -7,20 +7,19 @@
 // technical summary section 2) -- with an online softmax, so the cost is proportional to
 // the number of listed blocks.
 //
-// The listed key blocks are split between two softmax groups: group g takes the blocks at
-// list positions g, g+2, g+4, ... with its own S buffer, running max / sum, O accumulator
-// (all in TMEM) and P tile, and the two partial results are merged at the end.  The groups
-// run out of phase, so one group's exponentials (MUFU) overlap the other's max, P store
-// and waits, and the tensor core alternates between them.
+// Pipeline: S and P are double-buffered in TMEM (S_0, S_1, P_0, P_1, O = 512 columns), so
+// the MMA issuer computes S(t+2) = Q K_{t+2}^T as soon as the softmax has read S(t), and
+// O += P(t) V_t runs while the softmax works on block t+1: the softmax is the only serial
+// chain.
 //
 // Warp roles (352 threads):
 //   warp 0       TMA producer: Q tile once, then K_j tiles into a 3-slot ring;
 //   warp 10      TMA producer: V_j tiles into a 3-slot ring;
-//   warp 1       MMA issuer (one thread): S_g = Q K_j^T and O_g += P_g V_j (P_g read from
-//                TMEM, where it replaces S_g); owns TMEM;
-//   warps 2..5   softmax group 0, warps 6..9 softmax group 1: one query row per thread
-//                (TMEM lane = row); rescale O_g in TMEM only when the running max grows by
-//                more than 2^8; merge, normalise and store O and LSE at the end.
+//   warp 1       MMA issuer (one thread): S_b = Q K_j^T and O += P_b V_j (P_b read from
+//                TMEM); owns TMEM;
+//   warps 2..9   softmax + epilogue: thread = (query row, column half); warps w and w+4 share
+//                a TMEM lane quarter and exchange the row max once per key block; O is
+//                rescaled in TMEM only when the running max grows by more than 2^8.
 //
 // Shared-memory operands use the 128-byte swizzle that TMA writes: a 64-element (128 B)
 // slice of each row, eight rows per 1024-byte atom.  Q and K are K-major; V is read
@@ -51,8 +50,7 @@ __device__ unsigned long long g_trace[kTraceCtas][kTraceSlots];
 
 constexpr int BM = 128;            // query rows per MMA tile (TMEM lanes)
 constexpr int kSoftmaxWarp0 = 2;
-constexpr int kGroupWarps = 4;     // one warp per TMEM lane quarter
-constexpr int kSoftmaxWarps = 2 * kGroupWarps;
+constexpr int kSoftmaxWarps = 8;   // two warps per TMEM lane quarter: one per column half
 constexpr int kVWarp = kSoftmaxWarp0 + kSoftmaxWarps;   // V producer, after the softmax warps
 constexpr int kThreads = 32 * (kVWarp + 1);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when max grows > 2^8
@@ -81,20 +79,21 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-  // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], and per group
-  // s_full, p_full, o_done; final (MMA drain); merge (both groups' statistics)
+  // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2],
+  // s_free[2], p_full[2], o_done[2] (P*V done, per P buffer), final, pair[4 quarters][2 slots]
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST, B_VE = B_VF + VST,
-                       B_SF = B_VE + VST, B_P = B_SF + 2, B_O = B_P + 2,
-                       B_FIN = B_O + 2, B_MERGE = B_FIN + 1, NUM_BARS = B_MERGE + 1;
+                       B_SF = B_VE + VST, B_SE = B_SF + 2, B_P = B_SE + 2, B_O = B_P + 2,
+                       B_FIN = B_O + 2, B_PAIR = B_FIN + 1, NUM_BARS = B_PAIR + 8;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  // per-row statistics of each group for the merge: [group][m, l][BM] floats
+  // row-max / row-sum exchange between the column halves: [2 slots][2 halves][BM] floats
   static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
   // At least 120 KB so that one CTA (and one 512-column TMEM allocation) is resident per SM.
   static constexpr int SMEM_RAW = OFF_RED + 2 * 2 * BM * 4;
   static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-  // S_g at column 128 g (P_g, bf16, overwrites its first BN/2 columns), O_g at 256 + 128 g
-  static constexpr uint32_t TM_S = 0, TM_O = 256;
+  // TMEM columns: S_b at 128 b, P_b (bf16 pairs) at 256 + 64 b, O at 384
+  static constexpr uint32_t TM_S = 0, TM_P = 256, TM_O = 384;
+  static_assert(D <= 128 && BN <= 128, "TMEM layout");
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
 };
@@ -138,11 +137,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   auto bar_k_empty = [&](int s) { return bar0 + 8u * (C::B_KE + s); };
   auto bar_v_full = [&](int s) { return bar0 + 8u * (C::B_VF + s); };
   auto bar_v_empty = [&](int s) { return bar0 + 8u * (C::B_VE + s); };
-  auto bar_s_full = [&](int g) { return bar0 + 8u * (C::B_SF + g); };
-  auto bar_p_full = [&](int g) { return bar0 + 8u * (C::B_P + g); };
-  auto bar_o_done = [&](int g) { return bar0 + 8u * (C::B_O + g); };
+  auto bar_s_full = [&](int b) { return bar0 + 8u * (C::B_SF + b); };
+  auto bar_s_free = [&](int b) { return bar0 + 8u * (C::B_SE + b); };
+  auto bar_p_full = [&](int b) { return bar0 + 8u * (C::B_P + b); };
+  auto bar_o_done = [&](int b) { return bar0 + 8u * (C::B_O + b); };
   const uint32_t bar_final = bar0 + 8u * C::B_FIN;
-  const uint32_t bar_merge = bar0 + 8u * C::B_MERGE;
+  auto bar_pair = [&](int q, int slot) { return bar0 + 8u * (C::B_PAIR + 2 * q + slot); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   // Stays zero: the drain waits after an abort are bounded by time alone.
@@ -168,13 +168,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     mbar_init(bar_q, 1);
     for (int s = 0; s < C::KST; ++s) { mbar_init(bar_k_full(s), 1); mbar_init(bar_k_empty(s), 1); }
     for (int s = 0; s < C::VST; ++s) { mbar_init(bar_v_full(s), 1); mbar_init(bar_v_empty(s), 1); }
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(bar_s_full(g), 1);
-      mbar_init(bar_p_full(g), kGroupWarps);
-      mbar_init(bar_o_done(g), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_s_full(b), 1);
+      mbar_init(bar_s_free(b), kSoftmaxWarps);
+      mbar_init(bar_p_full(b), kSoftmaxWarps);
+      mbar_init(bar_o_done(b), 1);
     }
     mbar_init(bar_final, 1);
-    mbar_init(bar_merge, kSoftmaxWarps);
+    for (int q = 0; q < 4; ++q) { mbar_init(bar_pair(q, 0), 2); mbar_init(bar_pair(q, 1), 2); }
     *abort_flag = 0;
     *never = 0;
     mbar_fence_init();
@@ -226,52 +227,56 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Issue order: S(t) for group t&1, then O += P V for the block before it (other group).
-    // P_g lives in S_g's TMEM columns; the tensor core executes this thread's MMAs in
-    // order, so S(t+2) is written only after P(t) V has read P(t).
+    // S(t+2) is issued as soon as the softmax has read S(t) (same S buffer); O += P(t) V_t
+    // as soon as P(t) is in TMEM.  Descriptors are built once; an MMA only adds a byte
+    // offset / 16 to the start-address field (shared addresses stay below 2^18 bytes, so
+    // the 14-bit field never carries).
     if (lane == 0 && n > 0) {
-      // Descriptors are built once; an MMA only adds a byte offset / 16 to the start-address
-      // field (shared addresses stay below 2^18 bytes, so the 14-bit field never carries).
       const uint64_t q_desc = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t k_desc = smem_desc_sw128(sK, 16, 1024);
       const uint64_t v_desc = smem_desc_sw128(sV, BN * 128, 1024);
       bool ok = mbar_wait(bar_q, 0, abort_flag);
       bool any_mma = false;
-      auto issue_pv = [&](int t) -> bool {
-        const int g = t & 1, u = t >> 1, s = t % C::VST;
-        if (!mbar_wait(bar_p_full(g), u & 1, abort_flag)) return false;
-        if (!mbar_wait(bar_v_full(s), (t / C::VST) & 1, abort_flag)) return false;
-        tc_fence_after();
-        LVA_TRACE_AT(1, t);
-        const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
-        const uint32_t o_tm = tmem + C::TM_O + 128 * g, p_tm = tmem + C::TM_S + 128 * g;
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_f16_ts(o_tm, p_tm + kk * 8, vs + uint64_t((kk * 16 * 128) >> 4), C::IDESC_PV,
-                      (u > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar_v_empty(s));
-        umma_commit(bar_o_done(g));
-        return true;
-      };
-      for (int t = 0; ok && t < n; ++t) {
-        const int s = t % C::KST, g = t & 1;
-        ok = mbar_wait(bar_k_full(s), (t / C::KST) & 1, abort_flag);
-        if (!ok) break;
+      auto issue_qk = [&](int t) -> bool {
+        const int s = t % C::KST, b = t & 1;
+        if (!mbar_wait(bar_k_full(s), (t / C::KST) & 1, abort_flag)) return false;
+        if (t >= 2 && !mbar_wait(bar_s_free(b), ((t >> 1) - 1) & 1, abort_flag)) return false;
         tc_fence_after();
         LVA_TRACE_AT(0, t);
         const uint64_t ks = k_desc + uint64_t((s * C::KV_BYTES) >> 4);
-        const uint32_t s_tm = tmem + C::TM_S + 128 * g;
+        const uint32_t s_tm = tmem + C::TM_S + 128 * b;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           umma_f16_ss(s_tm, q_desc + uint64_t(((kk / 4) * BM * 128 + (kk % 4) * 32) >> 4),
                       ks + uint64_t(((kk / 4) * BN * 128 + (kk % 4) * 32) >> 4), C::IDESC_QK,
                       kk > 0 ? 1u : 0u);
-        umma_commit(bar_s_full(g));
+        umma_commit(bar_s_full(b));
         umma_commit(bar_k_empty(s));
         any_mma = true;
-        if (t >= 1) ok = issue_pv(t - 1);
+        return true;
+      };
+      auto issue_pv = [&](int t) -> bool {
+        const int s = t % C::VST, b = t & 1;
+        if (!mbar_wait(bar_p_full(b), (t >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar_v_full(s), (t / C::VST) & 1, abort_flag)) return false;
+        tc_fence_after();
+        LVA_TRACE_AT(1, t);
+        const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
+        const uint32_t p_tm = tmem + C::TM_P + 64 * b;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          umma_f16_ts(tmem + C::TM_O, p_tm + kk * 8, vs + uint64_t((kk * 16 * 128) >> 4), C::IDESC_PV,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar_v_empty(s));
+        umma_commit(bar_o_done(b));
+        return true;
+      };
+      if (ok) ok = issue_qk(0);
+      if (ok && n > 1) ok = issue_qk(1);
+      for (int t = 0; ok && t < n; ++t) {
+        if (t + 2 < n) ok = issue_qk(t + 2);
+        if (ok) ok = issue_pv(t);
       }
-      if (ok) ok = issue_pv(n - 1);
       if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 2); }
       if (any_mma) {
         // Drain: every MMA issued by this thread completes before TMEM is released.
@@ -280,76 +285,99 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax groups + epilogue
-    const int g = (warp - kSoftmaxWarp0) / kGroupWarps;   // group: list positions g, g+2, ...
+    // ------------------------------------------------------------ softmax + epilogue
+    // Thread = (query row, column half).  Warps w and w+4 share a TMEM lane quarter, so they
+    // own the same 32 rows; the first takes key/O columns [0, half), the second the rest.
+    constexpr int HALF = BN / 2, DH = D / 2;
+    const int hf = (warp - kSoftmaxWarp0) >> 2;   // column half
     const int sub = warp & 3;                     // TMEM lane quarter this warp may access
     const int row = sub * 32 + lane;              // row of the 128-row tile
     const uint32_t lane_off = uint32_t(sub * 32) << 16;
-    const uint32_t tS = tmem + lane_off + C::TM_S + 128 * g;
-    const uint32_t tO = tmem + lane_off + C::TM_O + 128 * g;
+    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);   // [slot][half][row]
+    // Exchange of one value per row with the partner warp (other column half).  Exchange
+    // number `seq` uses slot seq & 1; the partner's read of a slot always precedes its
+    // arrival on the next exchange, so a slot is never overwritten before it is read.
+    auto pair_exchange = [&](int seq, float v, bool& good) -> float {
+      float* slot = red + (seq & 1) * 2 * BM;
+      slot[hf * BM + row] = v;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_pair(sub, seq & 1));
+      good = __all_sync(0xffffffffu, mbar_wait(bar_pair(sub, seq & 1), (seq >> 1) & 1, abort_flag));
+      return good ? slot[(1 - hf) * BM + row] : 0.f;
+    };
     const float c = p.scale_log2;                 // scores -> log2 units
-    const int ng = n > g ? (n - g + 1) / 2 : 0;   // blocks of this group
     float m_ref = -INFINITY;                      // running max in log2 units (lazy)
-    float l = 0.f;
+    float l = 0.f;                                // this half's share of the row sum
     bool ok = true;
+    const bool tr = (sub == 2 && lane == 0 && hf == 0);
     if (bad && threadIdx.x == kSoftmaxWarp0 * 32) report_fault(p.err, 1, int(csr & 0x7fffffff));
-    int32_t jn = ng > 0 ? __ldg(p.col_idx + start + g) : 0;
+    int32_t jn = n > 0 ? __ldg(p.col_idx + start) : 0;
 
-    const bool tr = (sub == 2 && lane == 0);     // first warp of the group traces
-    for (int u = 0; u < ng; ++u) {
-      const int t = 2 * u + g;
+    for (int t = 0; t < n; ++t) {
+      const int b = t & 1;
       const int32_t j = jn;
-      if (u + 1 < ng) jn = __ldg(p.col_idx + start + t + 2);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(g), u & 1, abort_flag))) { ok = false; break; }
+      if (t + 1 < n) jn = __ldg(p.col_idx + start + t + 1);
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), (t >> 1) & 1, abort_flag))) { ok = false; break; }
       tc_fence_after();
-      if (tr) LVA_TRACE_AT(2 + 6 * g, t);
-      uint32_t sr[BN];
+      if (tr) LVA_TRACE_AT(2, t);
+      uint32_t sr[HALF];
 #pragma unroll
-      for (int q = 0; q < BN / 32; ++q)
-        tmem_ld32(tS + q * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
+      for (int q = 0; q < HALF / 32; ++q)
+        tmem_ld32(tmem + lane_off + C::TM_S + 128 * b + hf * HALF + q * 32,
+                  *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
       tmem_wait_ld();
-      if (tr) LVA_TRACE_AT(3 + 6 * g, t);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_s_free(b));
+      if (tr) LVA_TRACE_AT(3, t);
 
-      // Real keys of this block (only the block holding the sequence end is partial).
-      const int64_t valid = p.n_valid - int64_t(j) * BN;
+      // Real keys of this half (only the block holding the sequence end is partial).
+      const int64_t valid = p.n_valid - int64_t(j) * BN - hf * HALF;
       float mx;
-      if (valid >= BN) {
+      if (valid >= HALF) {
         // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (3-input max, 4 chains)
         float m4[4];
         if (c >= 0.f) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < BN / 2; ++e)
+          for (int e = 0; e < HALF / 2; ++e)
             m4[e & 3] = fmax3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
           mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
         } else {
 #pragma unroll
           for (int e = 0; e < 4; ++e) m4[e] = INFINITY;
 #pragma unroll
-          for (int e = 0; e < BN / 2; ++e)
+          for (int e = 0; e < HALF / 2; ++e)
             m4[e & 3] = fmin3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
           mx = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3])) * c;
         }
       } else {
         mx = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < BN; ++e)
+        for (int e = 0; e < HALF; ++e)
           if (e < valid) mx = fmaxf(mx, __uint_as_float(sr[e]) * c);
+      }
+      // Row max over both halves.
+      {
+        bool good;
+        const float other = pair_exchange(t, mx, good);
+        if (!good) { ok = false; break; }
+        mx = fmaxf(mx, other);
       }
       const float m_old = m_ref;
       if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
       const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       float r4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[BN / 2];
-      if (valid >= BN) {
+      uint32_t pk[HALF / 2];
+      if (valid >= HALF) {
         // Pairs of elements with packed fp32 math; every third pair takes its exponentials
         // on the FMA pipe, the rest on the MUFU, which balances the two units.
         const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
         uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
-        for (int e = 0; e < BN / 2; ++e) {
+        for (int e = 0; e < HALF / 2; ++e) {
           const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
           uint64_t p2;
           if (e % 3 == 2) {
@@ -370,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         r4[0] = a0; r4[1] = a1; r4[2] = b0; r4[3] = b1;
       } else {
 #pragma unroll
-        for (int e = 0; e < BN; e += 2) {
+        for (int e = 0; e < HALF; e += 2) {
           const float p0 = e < valid ? ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use)) : 0.f;
           const float p1 = e + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use)) : 0.f;
           r4[(e >> 1) & 3] += p0 + p1;
@@ -378,93 +406,87 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         }
       }
       l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
-      if (tr) LVA_TRACE_AT(4 + 6 * g, t);
+      if (tr) LVA_TRACE_AT(4, t);
 
-      // O_g may be rescaled only after this group's previous P*V has completed; without a
-      // rescale the next P*V simply follows it on the tensor pipe.
-      if (u >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(g), (u - 1) & 1, abort_flag))) { ok = false; break; }
+      // P_b was last read by O += P(t-2) V; O itself by O += P(t-1) V.  Each P buffer has
+      // its own completion barrier, so these waits never alias an older phase.
+      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), ((t >> 1) - 1) & 1, abort_flag))) {
+        ok = false; break;
+      }
+      if (t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(b ^ 1), ((t - 1) >> 1) & 1, abort_flag))) {
+          ok = false; break;
+        }
         tc_fence_after();
-        if (tr) LVA_TRACE_AT(5 + 6 * g, t);
+        if (tr) LVA_TRACE_AT(5, t);
 #pragma unroll 1
-        for (int q = 0; q < D / 32; ++q) {
+        for (int q = 0; q < DH / 32; ++q) {
           uint32_t ov[32];
-          tmem_ld32(tO + q * 32, ov);
+          tmem_ld32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(tO + q * 32, ov);
+          tmem_st32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
         }
       }
-      // P row (bf16 pairs) -> TMEM over the first BN/2 columns of S_g, the A operand of P*V.
+      tc_fence_after();
+      // P half row (bf16 pairs) -> TMEM P_b, the A operand of O += P V.
 #pragma unroll
-      for (int q = 0; q < BN / 64; ++q)
-        tmem_st32(tS + q * 32, *reinterpret_cast<const uint32_t(*)[32]>(pk + q * 32));
+      for (int q = 0; q < HALF / 64; ++q)
+        tmem_st32(tmem + lane_off + C::TM_P + 64 * b + hf * (HALF / 2) + q * 32,
+                  *reinterpret_cast<const uint32_t(*)[32]>(pk + q * 32));
+      if constexpr (HALF % 64 != 0) {
+        // BN = 64: a half row is 32 keys = 16 columns
+        tmem_st16(tmem + lane_off + C::TM_P + 64 * b + hf * (HALF / 2),
+                  *reinterpret_cast<const uint32_t(*)[16]>(pk));
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p_full(g));
-      if (tr) LVA_TRACE_AT(7 + 6 * g, t);
+      if (lane == 0) mbar_arrive(bar_p_full(b));
+      if (tr) LVA_TRACE_AT(7, t);
     }
 
-    // ------------------------------------------------------------ merge + epilogue
-    if (tr) LVA_TRACE_AT(16 + g, 0);
-    if (ok && ng > 0) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(g), (ng - 1) & 1, abort_flag))) ok = false;
+    // ------------------------------------------------------------ epilogue
+    if (tr) LVA_TRACE_AT(16, 0);
+    if (ok && n > 0) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag))) ok = false;
       else tc_fence_after();
     }
     if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 3); }
-    // Publish this group's (max, sum) per row; read the other group's.
-    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);      // [group][m, l][row]
-    red[(2 * g) * BM + row] = m_ref;
-    red[(2 * g + 1) * BM + row] = ok ? l : 0.f;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar_merge);
-    if (!__all_sync(0xffffffffu, mbar_wait(bar_merge, 0, abort_flag))) {
-      ok = false; *abort_flag = 1; report_fault(p.err, 5, 4);
+    // Row sum over both halves (exchange number n, after the n row-max exchanges).
+    float l_row = l;
+    if (ok && n > 0) {
+      bool good;
+      const float other = pair_exchange(n, l, good);
+      if (!good) { ok = false; *abort_flag = 1; report_fault(p.err, 5, 4); }
+      l_row += other;
     }
-    float m0 = red[0 * BM + row], l0 = red[1 * BM + row];
-    float m1 = red[2 * BM + row], l1 = red[3 * BM + row];
-    if (!ok) { l0 = 0.f; l1 = 0.f; }
-    const float m = fmaxf(m0, m1);
-    const float a0 = l0 > 0.f ? ex2_approx(m0 - m) : 0.f;     // weights of the two partials
-    const float a1 = l1 > 0.f ? ex2_approx(m1 - m) : 0.f;
-    const float lt = a0 * l0 + a1 * l1;
-    const bool have = lt > 0.f;
-    const float w0 = have ? a0 / lt : 0.f, w1 = have ? a1 / lt : 0.f;
-    const bool use0 = ok && n > 0 && l0 > 0.f, use1 = ok && n > 1 && l1 > 0.f;
-
-    // Each group normalises and stores half of the O columns of its rows.
-    constexpr int DH = D / 2;
     const int64_t grow = int64_t(i) * BN + row;           // row within the plane
     const bool store = row < BN && grow < p.n_pad;
-    __nv_bfloat16* orow = p.o + (plane * p.n_pad + grow) * D + g * DH;
-    const uint32_t tO0 = tmem + lane_off + C::TM_O + g * DH, tO1 = tO0 + 128;
+    const bool have = ok && n > 0 && l_row > 0.f;
+    const float inv_l = have ? 1.f / l_row : 0.f;
+    __nv_bfloat16* orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
 #pragma unroll 1
     for (int q = 0; q < DH / 32; ++q) {
-      uint32_t o0[32], o1[32];
+      uint32_t ov[32];
       if (ok && n > 0) {
-        tmem_ld32(tO0 + q * 32, o0);
-        if (n > 1) tmem_ld32(tO1 + q * 32, o1);
+        tmem_ld32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
         tmem_wait_ld();
       }
       uint32_t w[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        float x0 = 0.f, x1 = 0.f;
-        if (use0) { x0 = __uint_as_float(o0[2 * e]) * w0; x1 = __uint_as_float(o0[2 * e + 1]) * w0; }
-        if (use1) { x0 += __uint_as_float(o1[2 * e]) * w1; x1 += __uint_as_float(o1[2 * e + 1]) * w1; }
-        w[e] = pack_bf16x2(x0, x1);
-      }
+      for (int e = 0; e < 16; ++e)
+        w[e] = have ? pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l) : 0u;
       if (store) {
         uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
         for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
       }
     }
-    if (tr) LVA_TRACE_AT(18 + g, 0);
-    if (store && g == 0)
-      p.lse[plane * p.n_pad + grow] = have ? (m + __log2f(lt)) * 0.69314718055994530942f : -INFINITY;
+    if (tr) LVA_TRACE_AT(18, 0);
+    if (store && hf == 0)
+      p.lse[plane * p.n_pad + grow] = have ? (m_ref + __log2f(l_row)) * 0.69314718055994530942f : -INFINITY;
   }
 
   tc_fence_before();
