@@ -14,7 +14,10 @@ It is a plain, slow, obviously-correct restatement of what the hot path computes
                    matrices, and their per-query-block CSR lists;
 * ``attention`` -- masked softmax attention in float64, both block-wise (rows of one
                    query block share their key set) and by brute force over an explicit
-                   token-level mask.
+                   token-level mask;
+* ``calib``     -- the offline calibration of static masks: block energies of dense
+                   softmax attention, the minimal-prefix selection reaching a cumulative
+                   energy threshold, and the cross-prompt agreement threshold.
 
 Every function is pinned by tests under ``-m "not gpu"`` against hand-worked examples,
 closed forms, library routines and invariants; none is "parity unpinned".

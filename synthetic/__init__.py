@@ -5,8 +5,8 @@ the random static block masks that stand in for calibrated masks.  It contains
 none of the attention, reordering or mask-construction arithmetic; both the CUDA
 path and the FP64 oracle receive what it produces as plain inputs.
 """
-from .workloads import (WORKLOADS, Workload, make_qkv, mask_variants, spatial_repetition_map,
-                        static_calibrated_mask)
+from .workloads import (WORKLOADS, Workload, make_qk_calibration, make_qkv, mask_variants,
+                        spatial_repetition_map, static_calibrated_mask)
 
-__all__ = ["WORKLOADS", "Workload", "make_qkv", "static_calibrated_mask", "mask_variants",
-           "spatial_repetition_map"]
+__all__ = ["WORKLOADS", "Workload", "make_qkv", "make_qk_calibration", "static_calibrated_mask",
+           "mask_variants", "spatial_repetition_map"]

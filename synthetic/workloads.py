@@ -106,6 +106,38 @@ def make_qkv(w: Workload, heads: Optional[Iterable[int]] = None, dtype=torch.bfl
     return tuple(out)
 
 
+def make_qk_calibration(w: Workload, prompt: int, heads: Optional[Iterable[int]] = None,
+                        strength: float = 9.0, length_scale: float = 0.15,
+                        dtype=torch.bfloat16):
+    """Raster-order Q, K [B, H, n_valid, d] with space-time locality, one draw per prompt.
+
+    Stand-in for the activations of a video DiT during calibration (which needs trained
+    weights): every head has a fixed positional field F_h -- random Fourier features of the
+    normalised token position (t/T, y/Hg, x/Wg), F = sqrt(2/d) cos(W p + b) with W ~ N(0,
+    1/length_scale^2) and b ~ U[0, 2 pi), seeded by the workload and the head only -- and
+    each prompt adds its own N(0, 1) noise:  Q = strength * F + noise_q, K = strength * F +
+    noise_k.  <F_r, F_c> approximates exp(-|p_r - p_c|^2 / (2 length_scale^2)), so nearby
+    tokens score higher, and the structure is shared by all prompts while the noise is not.
+    """
+    hs = list(range(w.H)) if heads is None else list(heads)
+    t, y, x = torch.meshgrid(torch.arange(w.T), torch.arange(w.Hg), torch.arange(w.Wg), indexing="ij")
+    pos = torch.stack([t.reshape(-1) / max(1, w.T), y.reshape(-1) / max(1, w.Hg),
+                       x.reshape(-1) / max(1, w.Wg)], dim=1).to(torch.float64)      # [N, 3]
+    q = torch.empty((w.B, len(hs), w.n_valid, w.d), dtype=dtype)
+    k = torch.empty_like(q)
+    for hi, h in enumerate(hs):
+        g = _head_generator(w.seed, 7, 0, h)
+        freq = torch.randn((3, w.d), generator=g, dtype=torch.float64) / length_scale
+        phase = torch.rand((w.d,), generator=g, dtype=torch.float64) * (2 * math.pi)
+        field = (math.sqrt(2.0 / w.d) * torch.cos(pos @ freq + phase)).to(torch.float32)
+        for b in range(w.B):
+            gq = _head_generator(w.seed + 1_000 * (prompt + 1), 8, b, h)
+            gk = _head_generator(w.seed + 1_000 * (prompt + 1), 9, b, h)
+            q[b, hi] = (strength * field + torch.randn((w.n_valid, w.d), generator=gq)).to(dtype)
+            k[b, hi] = (strength * field + torch.randn((w.n_valid, w.d), generator=gk)).to(dtype)
+    return q, k
+
+
 def static_calibrated_mask(w: Workload, density: float = 0.30, seed_base: int = 1000) -> np.ndarray:
     """Random per-head static block mask [H, nb, nb] (uint8) standing in for a calibrated mask.
 
