@@ -33,34 +33,38 @@ import numpy as np
 from .attention import _as_f64
 
 
-def block_energy(q, k, block_size: int, n_valid: int, scale: float) -> np.ndarray:
+def block_energy(q, k, block_size: int, n_valid: int, scale: float, query_blocks=None) -> np.ndarray:
     """Block energies E [B, H, nb, nb] (float64) of dense softmax attention.
 
     q, k: [B, H, n_pad, d] (bf16-valued); ``scale`` is the caller's float32 value.
     Query block by query block: scores against every real key, the row softmax, then the
-    sum of the probabilities inside each key block.
+    sum of the probabilities inside each key block.  ``query_blocks`` optionally restricts
+    the work to a list of (b, h, i) triples; rows not computed are left as NaN.
     """
     q, k = _as_f64(q), _as_f64(k)
     B, H, n_pad, d = q.shape
     bs = block_size
     nb = n_pad // bs
     sc = float(np.float32(scale))
-    energy = np.zeros((B, H, nb, nb))
-    for b in range(B):
-        for h in range(H):
-            keys = k[b, h, :n_valid]
-            for i in range(nb):
-                r0, r1 = i * bs, min((i + 1) * bs, n_valid)
-                if r1 <= r0:
-                    continue                                   # padding rows only
-                s = sc * (q[b, h, r0:r1] @ keys.T)             # [rows, n_valid]
-                m = s.max(axis=1, keepdims=True)
-                e = np.exp(s - m)
-                a = e / e.sum(axis=1, keepdims=True)           # row softmax
-                for j in range(nb):
-                    c0, c1 = j * bs, min((j + 1) * bs, n_valid)
-                    if c1 > c0:
-                        energy[b, h, i, j] = a[:, c0:c1].sum()
+    if query_blocks is None:
+        energy = np.zeros((B, H, nb, nb))
+        query_blocks = [(b, h, i) for b in range(B) for h in range(H) for i in range(nb)]
+    else:
+        energy = np.full((B, H, nb, nb), np.nan)
+    for b, h, i in query_blocks:
+        energy[b, h, i] = 0.0
+        keys = k[b, h, :n_valid]
+        r0, r1 = i * bs, min((i + 1) * bs, n_valid)
+        if r1 <= r0:
+            continue                                           # padding rows only
+        s = sc * (q[b, h, r0:r1] @ keys.T)                     # [rows, n_valid]
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        a = e / e.sum(axis=1, keepdims=True)                   # row softmax
+        for j in range(nb):
+            c0, c1 = j * bs, min((j + 1) * bs, n_valid)
+            if c1 > c0:
+                energy[b, h, i, j] = a[:, c0:c1].sum()
     return energy
 
 
