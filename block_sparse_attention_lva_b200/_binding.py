@@ -48,6 +48,10 @@ SIGNATURES = {
     "lva_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
                                        _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp, _c_int, _vp]),
     "lva_broadcast_blocks": (_c_int, [_vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _vp, _c_int, _vp]),
+    "lva_block_energy": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int, _c_int,
+                                  _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp]),
+    "lva_select_blocks": (_c_int, [_vp, _vp, _c_i64, _c_int, ctypes.c_double, _vp]),
+    "lva_aggregate_masks": (_c_int, [_vp, _vp, _c_int, _c_i64, ctypes.c_double, _vp]),
     "lva_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
 }
 
@@ -210,6 +214,47 @@ def lva_broadcast_blocks(o, lse, block_size: int, query_src):
     _check(lib.lva_broadcast_blocks(_ptr(o), _ptr(lse), B, H, n_pad, d, block_size, _ptr(query_src),
                                     query_src.shape[0], ctypes.c_void_p(_stream(o.device))))
     return o, lse
+
+
+def lva_block_energy(q, k, lse, energy, n_valid: int, block_size: int, row_ptr, col_idx,
+                     mask_heads: int, scale: float):
+    """Block energies [B, H, nb, nb] (fp32) of softmax attention, given the dense-pass LSE."""
+    import torch
+    B, H, n_pad, d = q.shape
+    for name, t in (("q", q), ("k", k)):
+        _cuda_tensor(t, name, torch.bfloat16)
+        _need(tuple(t.shape) == (B, H, n_pad, d), f"{name} must have shape {(B, H, n_pad, d)}")
+    nb = n_pad // block_size
+    _cuda_tensor(lse, "lse", torch.float32, B * H * n_pad)
+    _cuda_tensor(energy, "energy", torch.float32, B * H * nb * nb)
+    _cuda_tensor(row_ptr, "row_ptr", torch.int32, mask_heads * nb + 1)
+    _cuda_tensor(col_idx, "col_idx", torch.int32)
+    _check(lib.lva_block_energy(_ptr(q), _ptr(k), _ptr(lse), _ptr(energy), B, H, n_pad, n_valid, d,
+                                block_size, _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), mask_heads,
+                                ctypes.c_float(scale), ctypes.c_void_p(_stream(q.device))))
+    return energy
+
+
+def lva_select_blocks(energy, mask, eps: float):
+    """0/1 mask (uint8, same shape) of the fewest key blocks reaching ``eps`` of each row's
+    energy; the last axis is the key block axis."""
+    import torch
+    _cuda_tensor(energy, "energy", torch.float32)
+    _cuda_tensor(mask, "mask", torch.uint8, energy.numel())
+    nb = energy.shape[-1]
+    _check(lib.lva_select_blocks(_ptr(energy), _ptr(mask), energy.numel() // nb, nb, ctypes.c_double(eps),
+                                 ctypes.c_void_p(_stream(energy.device))))
+    return mask
+
+
+def lva_aggregate_masks(masks, out, rho: float):
+    """Blocks kept by at least a fraction ``rho`` of the prompt masks ``masks[P, ...]``."""
+    import torch
+    _cuda_tensor(masks, "masks", torch.uint8)
+    _cuda_tensor(out, "out", torch.uint8, masks[0].numel())
+    _check(lib.lva_aggregate_masks(_ptr(masks), _ptr(out), masks.shape[0], out.numel(), ctypes.c_double(rho),
+                                   ctypes.c_void_p(_stream(masks.device))))
+    return out
 
 
 def lva_device_error(stream=None):

@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "liblva.so")
 
-SOURCES = ["api.cu", "reorder.cu", "mask.cu", "attn.cu", "broadcast.cu"]
+SOURCES = ["api.cu", "reorder.cu", "mask.cu", "attn.cu", "broadcast.cu", "tmap.cu", "energy.cu", "calib.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

@@ -228,6 +228,63 @@ lva_status lva_broadcast_blocks(void* o, float* lse, int B, int H, int64_t n_pad
   return from_cuda(launch_broadcast(a, stream), "broadcast launch");
 }
 
+lva_status lva_block_energy(const void* q, const void* k, const float* lse, float* energy, int B,
+                            int H, int64_t n_pad, int64_t n_valid, int d, int block_size,
+                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_len,
+                            int mask_heads, float scale, cudaStream_t stream) {
+  if (B < 0 || H < 1) return fail(LVA_ERR_INVALID_ARG, "energy: need B >= 0 and H >= 1");
+  if (d != 64 && d != 128) return fail(LVA_ERR_UNSUPPORTED, "energy: head dim must be 64 or 128");
+  if (block_size != 64 && block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "energy: block_size must be 64 or 128");
+  if (n_pad <= 0 || n_pad % block_size != 0) return fail(LVA_ERR_INVALID_ARG, "energy: n_pad must be a positive multiple of block_size");
+  if (n_valid < 0 || n_valid > n_pad) return fail(LVA_ERR_INVALID_ARG, "energy: need 0 <= n_valid <= n_pad");
+  if (mask_heads != 1 && mask_heads != H) return fail(LVA_ERR_INVALID_ARG, "energy: mask_heads must be 1 or H");
+  if (int64_t(B) * H * n_pad >= (int64_t(1) << 31)) return fail(LVA_ERR_UNSUPPORTED, "energy: B*H*n_pad must be < 2^31");
+  if (!(scale == scale)) return fail(LVA_ERR_INVALID_ARG, "energy: scale is NaN");
+  if (col_len < 0) return fail(LVA_ERR_INVALID_ARG, "energy: col_len < 0");
+  if (B == 0) return ok();
+  if (!q || !k || !lse || !energy || !row_ptr || (!col_idx && col_len > 0))
+    return fail(LVA_ERR_INVALID_ARG, "energy: null pointer");
+  if (!aligned(q, 16) || !aligned(k, 16))
+    return fail(LVA_ERR_INVALID_ARG, "energy: q, k must be 16-byte aligned");
+  if (!aligned(lse, 4) || !aligned(energy, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4))
+    return fail(LVA_ERR_INVALID_ARG, "energy: lse, energy, row_ptr, col_idx must be 4-byte aligned");
+  int* err = device_error_word();
+  if (err == nullptr) return fail(LVA_ERR_CUDA, "energy: cannot locate the device error word");
+  EnergyArgs a{q, k, lse, energy, B, H, n_pad, n_valid, d, block_size, row_ptr, col_idx, col_len,
+               mask_heads, scale, err};
+  const char* why = "launch";
+  cudaError_t e = launch_energy(a, stream, &why);
+  if (e != cudaSuccess) return fail(LVA_ERR_CUDA, "energy: %s: %s", why, cudaGetErrorString(e));
+  return ok();
+}
+
+lva_status lva_select_blocks(const float* energy, uint8_t* mask, int64_t rows, int nb, double eps,
+                             cudaStream_t stream) {
+  if (rows < 0) return fail(LVA_ERR_INVALID_ARG, "select: rows < 0");
+  if (nb < 1) return fail(LVA_ERR_INVALID_ARG, "select: nb must be >= 1");
+  if (nb > kSelectMaxBlocks) return fail(LVA_ERR_UNSUPPORTED, "select: nb must be <= %d", kSelectMaxBlocks);
+  if (!(eps >= 0.0 && eps <= 1.0)) return fail(LVA_ERR_INVALID_ARG, "select: eps must be in [0, 1]");
+  if (rows > (int64_t(1) << 40) / nb) return fail(LVA_ERR_UNSUPPORTED, "select: rows * nb too large");
+  if (rows == 0) return ok();
+  if (!energy || !mask) return fail(LVA_ERR_INVALID_ARG, "select: null pointer");
+  if (!aligned(energy, 4)) return fail(LVA_ERR_INVALID_ARG, "select: energy must be 4-byte aligned");
+  int* err = device_error_word();
+  if (err == nullptr) return fail(LVA_ERR_CUDA, "select: cannot locate the device error word");
+  SelectArgs a{energy, mask, rows, nb, eps, err};
+  return from_cuda(launch_select(a, stream), "select launch");
+}
+
+lva_status lva_aggregate_masks(const uint8_t* masks, uint8_t* out, int prompts, int64_t count,
+                               double rho, cudaStream_t stream) {
+  if (prompts < 1) return fail(LVA_ERR_INVALID_ARG, "aggregate: prompts must be >= 1");
+  if (count < 0) return fail(LVA_ERR_INVALID_ARG, "aggregate: count < 0");
+  if (!(rho >= 0.0 && rho <= 1.0)) return fail(LVA_ERR_INVALID_ARG, "aggregate: rho must be in [0, 1]");
+  if (count == 0) return ok();
+  if (!masks || !out) return fail(LVA_ERR_INVALID_ARG, "aggregate: null pointer");
+  AggregateArgs a{masks, out, prompts, count, rho * double(prompts)};
+  return from_cuda(launch_aggregate(a, stream), "aggregate launch");
+}
+
 lva_status lva_device_error(cudaStream_t stream, lva_status* status, int* detail) {
   if (status == nullptr) return fail(LVA_ERR_INVALID_ARG, "device_error: null status");
   int* err = device_error_word();

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace lva {
@@ -64,6 +65,50 @@ struct BroadcastArgs {
   int* err;
 };
 cudaError_t launch_broadcast(const BroadcastArgs& a, cudaStream_t stream);
+
+struct EnergyArgs {
+  const void* q;
+  const void* k;
+  const float* lse;
+  float* energy;
+  int B, H;
+  int64_t n_pad, n_valid;
+  int d, block_size;
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  int64_t col_len;
+  int mask_heads;
+  float scale;
+  int* err;
+};
+cudaError_t launch_energy(const EnergyArgs& a, cudaStream_t stream, const char** why);
+
+struct SelectArgs {
+  const float* energy;   // [rows, nb]
+  uint8_t* mask;         // [rows, nb]
+  int64_t rows;
+  int nb;
+  double eps;
+  int* err;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+
+struct AggregateArgs {
+  const uint8_t* masks;  // [prompts, count]
+  uint8_t* out;          // [count]
+  int prompts;
+  int64_t count;
+  double threshold;      // rho * prompts, in float64
+};
+cudaError_t launch_aggregate(const AggregateArgs& a, cudaStream_t stream);
+
+// Largest nb the selection supports (its sort holds a row in shared memory).
+constexpr int kSelectMaxBlocks = 4096;
+
+// 2D tensor map over a bf16 [rows, d] row-major matrix, box of 64 elements x box_rows,
+// 128-byte swizzle (from tmap.cu).  Returns false when the driver entry point is missing
+// or the encoding fails.
+bool make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows);
 
 // Device error word of the current device (from api.cu).
 int* device_error_word();

@@ -200,3 +200,74 @@ class SquadTwoPass:
                                  self.n, self.block_size, rp, ci, 1, self.scale)
         self._transpose(self.o_t, self.o, P, inverse=True)
         return self.o
+
+
+class StaticMaskCalibrator:
+    """Offline calibration of a static block mask from calibration prompts, over the C ABI.
+
+    CalibAtt page ("Accelerating Text-to-Video Generation with Calibrated Sparse Attention"),
+    section 2 A.1-A.2, for one (timestep, layer): every calibration sample (a prompt, i.e.
+    one batch element of one ``add_prompt`` call) goes through
+
+    1. ``lva_reorder_tokens`` of Q and K into tile order;
+    2. ``lva_block_sparse_attn`` with the all-ones mask, for the row LSE of dense attention;
+    3. ``lva_block_energy`` -> E [B, H, nb, nb], the attention mass of every block pair;
+    4. ``lva_select_blocks`` with the timestep's threshold ``eps`` -> a 0/1 mask per sample;
+
+    and ``finish(rho)`` keeps the blocks that at least a fraction ``rho`` of the samples
+    selected (``lva_aggregate_masks``).  The result, uint8 [H, nb, nb] in tile order, is the
+    ``static_mask`` of ``VideoBlockSparseAttention`` with ``mask={"kind": "static"}``.
+    """
+
+    def __init__(self, B, H, d, grid, tile, block_size=128, scale=None, device="cuda"):
+        self.B, self.H, self.d = B, H, d
+        self.grid, self.tile, self.block_size = tuple(grid), tuple(tile), block_size
+        self.n_valid = grid[0] * grid[1] * grid[2]
+        self.n_pad = (self.n_valid + block_size - 1) // block_size * block_size
+        self.nb = self.n_pad // block_size
+        self.scale = float(scale) if scale is not None else float(torch.tensor(d ** -0.5, dtype=torch.float32))
+        self.device = torch.device(device)
+        kw = dict(device=self.device)
+        shape = (B, H, self.n_pad, d)
+        self.qk_t = torch.empty((2,) + shape, dtype=torch.bfloat16, **kw)
+        self.q_t, self.k_t = self.qk_t[0], self.qk_t[1]
+        self.o_t = torch.empty(shape, dtype=torch.bfloat16, **kw)     # dense-pass output, unused
+        self.lse = torch.empty((B, H, self.n_pad), dtype=torch.float32, **kw)
+        self.energy = torch.empty((B, H, self.nb, self.nb), dtype=torch.float32, **kw)
+        p = lb.MaskParams(lb.LVA_MASK_ALL, self.n_pad, self.n_valid, block_size, 1)
+        self.row_ptr = torch.empty(self.nb + 1, dtype=torch.int32, **kw)
+        self.col_idx = torch.empty(lb.lva_block_mask_max_nnz(p), dtype=torch.int32, **kw)
+        self.nnz = torch.empty(1, dtype=torch.int32, **kw)
+        lb.lva_build_block_mask(p, None, self.row_ptr, self.col_idx, self.nnz)
+        self.samples = []
+
+    def energies(self, q, k):
+        """Raster-order bf16 Q, K [B, H, N, d] -> block energies E [B, H, nb, nb] (tile order)."""
+        P = self.B * self.H
+        for src, dst in ((q, self.q_t), (k, self.k_t)):
+            lb.lva_reorder_tokens(src.reshape(P, self.n_valid, self.d), dst.view(P, self.n_pad, self.d),
+                                  self.grid, self.tile, self.n_pad, inverse=False)
+        # V only feeds the unused dense output; K stands in for it.
+        lb.lva_block_sparse_attn(self.q_t, self.k_t, self.k_t, self.o_t, self.lse, self.n_valid,
+                                 self.block_size, self.row_ptr, self.col_idx, 1, self.scale)
+        lb.lva_block_energy(self.q_t, self.k_t, self.lse, self.energy, self.n_valid, self.block_size,
+                            self.row_ptr, self.col_idx, 1, self.scale)
+        return self.energy
+
+    def add_prompt(self, q, k, eps: float):
+        """Select the blocks of every sample of this batch at threshold ``eps``; returns the
+        per-sample masks uint8 [B, H, nb, nb]."""
+        energy = self.energies(q, k)
+        mask = torch.empty(energy.shape, dtype=torch.uint8, device=self.device)
+        lb.lva_select_blocks(energy, mask, eps)
+        self.samples.append(mask)
+        return mask
+
+    def finish(self, rho: float):
+        """Aggregated static mask uint8 [H, nb, nb] over every sample added so far."""
+        if not self.samples:
+            raise ValueError("no calibration prompt was added")
+        masks = torch.cat(self.samples, dim=0).contiguous()            # [S, H, nb, nb]
+        out = torch.empty(masks.shape[1:], dtype=torch.uint8, device=self.device)
+        lb.lva_aggregate_masks(masks, out, rho)
+        return out

@@ -200,6 +200,69 @@ lva_status lva_broadcast_blocks(void* o, float* lse, int B, int H, int64_t n_pad
                                 cudaStream_t stream);
 
 /*
+ * lva_block_energy -- block energies of softmax attention (static-mask calibration).
+ *
+ * CalibAtt page ("Accelerating Text-to-Video Generation with Calibrated Sparse Attention",
+ * section 2 A.1): the attention matrix is divided into Bs x Bs blocks and, for every query
+ * block, the energy toward a key block is the sum of its attention scores.  For batch b,
+ * head h, query block i and each key block j listed in CSR row h_m*nb + i:
+ *   E[b][h][i][j] = sum over r in block i with r < n_valid, c in block j with c < n_valid of
+ *                   exp(scale * <q_r, k_c> - LSE[b][h][r])
+ * where LSE must be the row log-sum-exp over all real keys (what lva_block_sparse_attn
+ * returns with the all-ones mask); rows whose LSE is not finite contribute 0.  Key blocks not
+ * listed get E = 0, so the whole row E[b][h][i][0..nb) is written.  The sum of a row is the
+ * number of real query rows in block i (up to rounding).
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation, fp32 exponentials and sums
+ * in a fixed order (the result does not depend on timing).
+ *
+ * q, k: device bf16 [B, H, n_pad, d], 16-byte aligned; lse: device fp32 [B, H, n_pad];
+ * energy: device fp32 [B, H, nb, nb] (caller-owned, written).  row_ptr / col_idx / col_len /
+ * mask_heads: a CSR block list as for lva_block_sparse_attn (the all-ones list for a dense
+ * calibration pass).  Bad CSR rows are skipped (their energy row stays 0) and reported
+ * through lva_device_error as LVA_ERR_INVALID_ARG.
+ * Supported: d in {64, 128}, block_size in {64, 128}, B*H*n_pad < 2^31.
+ */
+lva_status lva_block_energy(const void* q, const void* k, const float* lse, float* energy, int B,
+                            int H, int64_t n_pad, int64_t n_valid, int d, int block_size,
+                            const int32_t* row_ptr, const int32_t* col_idx, int64_t col_len,
+                            int mask_heads, float scale, cudaStream_t stream);
+
+/*
+ * lva_select_blocks -- fewest key blocks reaching a cumulative energy threshold.
+ *
+ * CalibAtt page (section 2 A.1): for every query block, the minimum number of key blocks
+ * needed to reach the cumulative energy threshold eps(t) is selected (eps is higher early in
+ * denoising and lower late; the caller passes the value for the timestep).  For every row
+ * x of energy[rows][nb]:
+ *   order  = key blocks by descending energy, equal energies by ascending index;
+ *   S_k    = sum of the first k energies of that order, one float64 addition at a time;
+ *   k*     = the smallest k >= 0 with S_k >= eps * S_nb (float64 product);
+ *   mask[x][j] = 1 for the first k* blocks of the order, else 0.
+ * A row of zeros (a query block of padding rows) selects nothing; eps = 0 selects nothing.
+ *
+ * energy: device fp32 [rows, nb], finite and >= 0 (a row holding anything else selects
+ * nothing and is reported through lva_device_error as LVA_ERR_INVALID_ARG, detail = row).
+ * mask: device uint8 [rows, nb] (caller-owned, written).  eps in [0, 1].
+ * Supported: 1 <= nb <= 4096 (LVA_ERR_UNSUPPORTED beyond).
+ */
+lva_status lva_select_blocks(const float* energy, uint8_t* mask, int64_t rows, int nb, double eps,
+                             cudaStream_t stream);
+
+/*
+ * lva_aggregate_masks -- cross-prompt agreement of calibration masks.
+ *
+ * CalibAtt page (section 2 A.2): the masks of the calibration prompts are averaged and a
+ * block is kept only when it was selected in a large enough fraction rho of them, which gives
+ * one data-independent mask per (timestep, layer, head).  For x < count:
+ *   out[x] = 1 if (number of p < prompts with masks[p*count + x] != 0) >= rho * prompts
+ *            (compared in float64), else 0.
+ * masks: device uint8 [prompts, count]; out: device uint8 [count] (caller-owned, written).
+ * prompts >= 1, rho in [0, 1].  The result is the dense input of the STATIC mask kind.
+ */
+lva_status lva_aggregate_masks(const uint8_t* masks, uint8_t* out, int prompts, int64_t count,
+                               double rho, cudaStream_t stream);
+
+/*
  * lva_device_error -- read and clear the current device's kernel error word.
  *
  * Synchronises `stream`, then stores in *status the first kernel-side fault recorded since

@@ -91,3 +91,27 @@ def test_mask_capacity_check():
     vp = ctypes.c_void_p(64)
     assert lib.lva_build_block_mask(ctypes.byref(p), None, vp, vp, 63, vp, None) == 3
     assert b"col_capacity" in lib.lva_last_error_message()
+
+
+def test_calibration_argument_checks_fail_before_launch():
+    from block_sparse_attention_lva_b200._binding import lib
+    vp = ctypes.c_void_p(64)
+    energy = lambda **kw: lib.lva_block_energy(
+        kw.get("q", vp), vp, vp, vp, 1, 2, kw.get("n_pad", 256), kw.get("n_valid", 256), kw.get("d", 128),
+        kw.get("bs", 128), vp, vp, 4, kw.get("mh", 1), ctypes.c_float(0.1), None)
+    assert energy(d=96) == 2
+    assert energy(bs=32) == 2
+    assert energy(n_pad=200) == 1
+    assert energy(mh=3) == 1
+    assert energy(q=ctypes.c_void_p(72)) == 1      # not 16-byte aligned
+    assert energy(q=None) == 1
+    sel = lambda rows, nb, eps: lib.lva_select_blocks(vp, vp, rows, nb, ctypes.c_double(eps), None)
+    assert sel(4, 0, 0.5) == 1                     # no key blocks
+    assert sel(4, 5000, 0.5) == 2                  # beyond the supported row length
+    assert sel(4, 16, 1.5) == 1 and sel(4, 16, -0.1) == 1
+    assert sel(0, 16, 0.5) == 0                    # no rows: no-op
+    assert lib.lva_select_blocks(None, vp, 4, 16, ctypes.c_double(0.5), None) == 1
+    agg = lambda prompts, count, rho: lib.lva_aggregate_masks(vp, vp, prompts, count, ctypes.c_double(rho), None)
+    assert agg(0, 16, 0.5) == 1
+    assert agg(2, 16, 1.5) == 1
+    assert agg(2, 0, 0.5) == 0
