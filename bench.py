@@ -381,7 +381,7 @@ def run_report(args):
     burst, sustained, hbm, peak_kind = _peaks()
     names = args.report.split(",")
     for name in names:
-        if name in ("stress", "squad"):
+        if name in ("stress", "squad", "calib"):
             continue
         w = WORKLOADS[name]
         q, k, v = make_qkv(w)
@@ -450,6 +450,45 @@ def run_report(args):
               flush=True)
         del qkv, op
         torch.cuda.empty_cache()
+    # Static-mask calibration on the small workload (12 heads, 32,768 tokens, 256 x 256 blocks):
+    # the dense pass for LSE, the block energies of all 786,432 block pairs, the selection of
+    # 3,072 energy rows and the aggregation of 4 samples.
+    if "calib" in names:
+        from synthetic import make_qk_calibration
+        w = WORKLOADS["small"]
+        q, k = make_qk_calibration(w, prompt=0)
+        qd, kd = q.to(dev), k.to(dev)
+        cal = lva.StaticMaskCalibrator(w.B, w.H, w.d, (w.T, w.Hg, w.Wg), w.tile, w.block_size,
+                                       scale=w.scale, device=dev)
+        cal.energies(qd, kd)
+        ms_dense = _time_cuda(lambda: lva.lva_block_sparse_attn(
+            cal.q_t, cal.k_t, cal.k_t, cal.o_t, cal.lse, w.n_valid, w.block_size, cal.row_ptr, cal.col_idx, 1,
+            cal.scale))
+        ms_energy = _time_cuda(lambda: lva.lva_block_energy(
+            cal.q_t, cal.k_t, cal.lse, cal.energy, w.n_valid, w.block_size, cal.row_ptr, cal.col_idx, 1,
+            cal.scale))
+        mask = torch.empty(cal.energy.shape, dtype=torch.uint8, device=dev)
+        ms_select = _time_cuda(lambda: lva.lva_select_blocks(cal.energy, mask, 0.8))
+        samples = mask.unsqueeze(0).repeat(4, 1, 1, 1, 1).reshape(4, w.H, w.nb, w.nb).contiguous()
+        out = torch.empty((w.H, w.nb, w.nb), dtype=torch.uint8, device=dev)
+        ms_agg = _time_cuda(lambda: lva.lva_aggregate_masks(samples, out, 0.5))
+        ms_total = _time_cuda(lambda: cal.add_prompt(qd, kd, 0.8))
+        cal.samples.clear()
+        status, detail = lva.lva_device_error()
+        pairs = w.B * w.H * w.nb * w.nb
+        qk_flops = pairs * 2.0 * w.block_size * w.block_size * w.d
+        exps = pairs * float(w.block_size * w.block_size)
+        print(json.dumps({"report": "calibration", "workload": "small (12 heads, 32,768 tokens)",
+                          "block_pairs": pairs, "dense_attn_ms": ms_dense, "energy_ms": ms_energy,
+                          "energy_qk_tflops": qk_flops / ms_energy / 1e9,
+                          "energy_qk_frac_of_sustained": qk_flops / ms_energy / 1e9 / sustained,
+                          "energy_exp_per_s": exps / ms_energy * 1e3,
+                          "select_ms": ms_select, "select_rows": w.B * w.H * w.nb,
+                          "aggregate_ms": ms_agg, "aggregate_bytes": 5 * w.H * w.nb * w.nb,
+                          "add_prompt_ms": ms_total, "selected_density_eps0.8": float(mask.float().mean()),
+                          "kernel_error": status}), flush=True)
+        del qd, kd, cal, samples, out, mask
+        torch.cuda.empty_cache()
     # mask-builder stress size: static mask, 40 heads x 4096 x 4096 blocks (671 MB read)
     if "stress" in names or args.report_stress:
         hm, nb = 40, 4096
@@ -475,7 +514,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--report", default="", help="comma list of workloads (tiny,small,static,large,long,stress,squad): "
+    ap.add_argument("--report", default="", help="comma list of workloads (tiny,small,static,large,long,stress,squad,calib): "
                     "per-mask kernel timings and the density sweep fit instead of the bench line")
     ap.add_argument("--report-stress", action="store_true")
     args = ap.parse_args()
