@@ -12,13 +12,14 @@
 // O += P(t) V_t runs while the softmax works on block t+1: the softmax is the only serial
 // chain.
 //
-// Warp roles (352 threads):
+// Warp roles (384 threads):
 //   warp 0       TMA producer: Q tile once, then K_j tiles into a 3-slot ring;
 //   warp 10      TMA producer: V_j tiles into a 3-slot ring;
-//   warp 1       MMA issuer (one thread): S_b = Q K_j^T and O += P_b V_j (P_b read from
-//                TMEM); owns TMEM;
-//   warps 2..9   softmax + epilogue: thread = (query row, column half); warps w and w+4 share
-//                a TMEM lane quarter and exchange the row max once per key block; O is
+//   warp 1       MMA issuer (one thread): S_b = Q K_j^T; owns TMEM;
+//   warp 11      MMA issuer (one thread): O += P_b V_j (P_b read from TMEM);
+//   warps 2..9   softmax + epilogue: each warp owns 16 rows of the 128-row tile; lane t and
+//                lane t + 16 hold the left and right column halves of one row (the .16x32bx2
+//                TMEM shapes), so row maxima and sums meet through one shuffle; O is
 //                rescaled in TMEM only when the running max grows by more than 2^8.
 //
 // Shared-memory operands use the 128-byte swizzle that TMA writes: a 64-element (128 B)
@@ -50,9 +51,10 @@ __device__ unsigned long long g_trace[kTraceCtas][kTraceSlots];
 
 constexpr int BM = 128;            // query rows per MMA tile (TMEM lanes)
 constexpr int kSoftmaxWarp0 = 2;
-constexpr int kSoftmaxWarps = 8;   // two warps per TMEM lane quarter: one per column half
+constexpr int kSoftmaxWarps = 8;   // two warps per TMEM lane quarter: 16 rows each
 constexpr int kVWarp = kSoftmaxWarp0 + kSoftmaxWarps;   // V producer, after the softmax warps
-constexpr int kThreads = 32 * (kVWarp + 1);
+constexpr int kPVWarp = kVWarp + 1;                       // issuer of O += P V
+constexpr int kThreads = 32 * (kPVWarp + 1);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when max grows > 2^8
 constexpr uint32_t kTmemCols = 512;
 
@@ -80,15 +82,13 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
   // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2],
-  // s_free[2], p_full[2], o_done[2] (P*V done, per P buffer), final, pair[4 quarters][2 slots]
+  // s_free[2], p_full[2], o_done[2] (P*V done, per P buffer), final (Q K^T), final (P V)
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST, B_VE = B_VF + VST,
                        B_SF = B_VE + VST, B_SE = B_SF + 2, B_P = B_SE + 2, B_O = B_P + 2,
-                       B_FIN = B_O + 2, B_PAIR = B_FIN + 1, NUM_BARS = B_PAIR + 8;
+                       B_FIN = B_O + 2, B_FIN_PV = B_FIN + 1, NUM_BARS = B_FIN_PV + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  // row-max / row-sum exchange between the column halves: [2 slots][2 halves][BM] floats
-  static constexpr int OFF_RED = (OFF_MISC + 16 + 15) / 16 * 16;
   // At least 120 KB so that one CTA (and one 512-column TMEM allocation) is resident per SM.
-  static constexpr int SMEM_RAW = OFF_RED + 2 * 2 * BM * 4;
+  static constexpr int SMEM_RAW = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
   // TMEM columns: S_b at 128 b, P_b (bf16 pairs) at 256 + 64 b, O at 384
@@ -142,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   auto bar_p_full = [&](int b) { return bar0 + 8u * (C::B_P + b); };
   auto bar_o_done = [&](int b) { return bar0 + 8u * (C::B_O + b); };
   const uint32_t bar_final = bar0 + 8u * C::B_FIN;
-  auto bar_pair = [&](int q, int slot) { return bar0 + 8u * (C::B_PAIR + 2 * q + slot); };
+  const uint32_t bar_final_pv = bar0 + 8u * C::B_FIN_PV;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   // Stays zero: the drain waits after an abort are bounded by time alone.
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       mbar_init(bar_o_done(b), 1);
     }
     mbar_init(bar_final, 1);
-    for (int q = 0; q < 4; ++q) { mbar_init(bar_pair(q, 0), 2); mbar_init(bar_pair(q, 1), 2); }
+    mbar_init(bar_final_pv, 1);
     *abort_flag = 0;
     *never = 0;
     mbar_fence_init();
@@ -226,21 +226,21 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       produce(&tm_v, sV, C::VST, bar_v_full(0), bar_v_empty(0), 6);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // S(t+2) is issued as soon as the softmax has read S(t) (same S buffer); O += P(t) V_t
-    // as soon as P(t) is in TMEM.  Descriptors are built once; an MMA only adds a byte
-    // offset / 16 to the start-address field (shared addresses stay below 2^18 bytes, so
-    // the 14-bit field never carries).
+    // ------------------------------------------------------------ MMA issuer: S = Q K^T
+    // S(t+2) is issued as soon as the softmax has read S(t) (same S buffer).  O += P V is
+    // issued by its own warp, so neither issue stream waits behind the other's barriers;
+    // the two write disjoint TMEM columns and read disjoint shared memory.  Descriptors are
+    // built once; an MMA only adds a byte offset / 16 to the start-address field (shared
+    // addresses stay below 2^18 bytes, so the 14-bit field never carries).
     if (lane == 0 && n > 0) {
       const uint64_t q_desc = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t k_desc = smem_desc_sw128(sK, 16, 1024);
-      const uint64_t v_desc = smem_desc_sw128(sV, BN * 128, 1024);
       bool ok = mbar_wait(bar_q, 0, abort_flag);
       bool any_mma = false;
-      auto issue_qk = [&](int t) -> bool {
+      for (int t = 0; ok && t < n; ++t) {
         const int s = t % C::KST, b = t & 1;
-        if (!mbar_wait(bar_k_full(s), (t / C::KST) & 1, abort_flag)) return false;
-        if (t >= 2 && !mbar_wait(bar_s_free(b), ((t >> 1) - 1) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar_k_full(s), (t / C::KST) & 1, abort_flag)) { ok = false; break; }
+        if (t >= 2 && !mbar_wait(bar_s_free(b), ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         LVA_TRACE_AT(0, t);
         const uint64_t ks = k_desc + uint64_t((s * C::KV_BYTES) >> 4);
@@ -253,12 +253,24 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         umma_commit(bar_s_full(b));
         umma_commit(bar_k_empty(s));
         any_mma = true;
-        return true;
-      };
-      auto issue_pv = [&](int t) -> bool {
+      }
+      if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 2); }
+      if (any_mma) {
+        // Drain: every MMA issued by this thread completes before TMEM is released.
+        umma_commit(bar_final);
+        mbar_wait(bar_final, 0, never);
+      }
+    }
+  } else if (warp == kPVWarp) {
+    // ------------------------------------------------------------ MMA issuer: O += P V
+    // O += P(t) V_t as soon as P(t) is in TMEM and V_t has landed; P is the TMEM A operand.
+    if (lane == 0 && n > 0) {
+      const uint64_t v_desc = smem_desc_sw128(sV, BN * 128, 1024);
+      bool ok = true, any_mma = false;
+      for (int t = 0; ok && t < n; ++t) {
         const int s = t % C::VST, b = t & 1;
-        if (!mbar_wait(bar_p_full(b), (t >> 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(bar_v_full(s), (t / C::VST) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar_p_full(b), (t >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar_v_full(s), (t / C::VST) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         LVA_TRACE_AT(1, t);
         const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
@@ -269,47 +281,30 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
                       (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar_v_empty(s));
         umma_commit(bar_o_done(b));
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      if (ok && n > 1) ok = issue_qk(1);
-      for (int t = 0; ok && t < n; ++t) {
-        if (t + 2 < n) ok = issue_qk(t + 2);
-        if (ok) ok = issue_pv(t);
+        any_mma = true;
       }
-      if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 2); }
+      if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 7); }
       if (any_mma) {
-        // Drain: every MMA issued by this thread completes before TMEM is released.
-        umma_commit(bar_final);
-        mbar_wait(bar_final, 0, never);
+        umma_commit(bar_final_pv);
+        mbar_wait(bar_final_pv, 0, never);
       }
     }
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    // Thread = (query row, column half).  Warps w and w+4 share a TMEM lane quarter, so they
-    // own the same 32 rows; the first takes key/O columns [0, half), the second the rest.
+    // Thread = (query row, column half).  The warp may access TMEM lane quarter w & 3 and
+    // takes 16 of its 32 lanes; with the .16x32bx2 shapes lane t (t < 16) moves columns
+    // [0, half) of row base + t and lane t + 16 columns [half, 2 half) of the same row.
     constexpr int HALF = BN / 2, DH = D / 2;
-    const int hf = (warp - kSoftmaxWarp0) >> 2;   // column half
-    const int sub = warp & 3;                     // TMEM lane quarter this warp may access
-    const int row = sub * 32 + lane;              // row of the 128-row tile
-    const uint32_t lane_off = uint32_t(sub * 32) << 16;
-    float* red = reinterpret_cast<float*>(smem + C::OFF_RED);   // [slot][half][row]
-    // Exchange of one value per row with the partner warp (other column half).  Exchange
-    // number `seq` uses slot seq & 1; the partner's read of a slot always precedes its
-    // arrival on the next exchange, so a slot is never overwritten before it is read.
-    auto pair_exchange = [&](int seq, float v, bool& good) -> float {
-      float* slot = red + (seq & 1) * 2 * BM;
-      slot[hf * BM + row] = v;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_pair(sub, seq & 1));
-      good = __all_sync(0xffffffffu, mbar_wait(bar_pair(sub, seq & 1), (seq >> 1) & 1, abort_flag));
-      return good ? slot[(1 - hf) * BM + row] : 0.f;
-    };
+    const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
+    const int sel = (warp - kSoftmaxWarp0) >> 2;  // which 16 lanes of the quarter
+    const int hf = lane >> 4;                     // column half
+    const int row = quarter * 32 + sel * 16 + (lane & 15);   // row of the 128-row tile
+    const uint32_t lane_off = uint32_t(quarter * 32 + sel * 16) << 16;
     const float c = p.scale_log2;                 // scores -> log2 units
     float m_ref = -INFINITY;                      // running max in log2 units (lazy)
     float l = 0.f;                                // this half's share of the row sum
     bool ok = true;
-    const bool tr = (sub == 2 && lane == 0 && hf == 0);
+    const bool tr = (quarter == 2 && sel == 0 && lane == 0);
     if (bad && threadIdx.x == kSoftmaxWarp0 * 32) report_fault(p.err, 1, int(csr & 0x7fffffff));
     int32_t jn = n > 0 ? __ldg(p.col_idx + start) : 0;
 
@@ -323,8 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       uint32_t sr[HALF];
 #pragma unroll
       for (int q = 0; q < HALF / 32; ++q)
-        tmem_ld32(tmem + lane_off + C::TM_S + 128 * b + hf * HALF + q * 32,
-                  *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
+        tmem_ld_16x2_32<HALF>(tmem + lane_off + C::TM_S + 128 * b + q * 32,
+                              *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -358,13 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         for (int e = 0; e < HALF; ++e)
           if (e < valid) mx = fmaxf(mx, __uint_as_float(sr[e]) * c);
       }
-      // Row max over both halves.
-      {
-        bool good;
-        const float other = pair_exchange(t, mx, good);
-        if (!good) { ok = false; break; }
-        mx = fmaxf(mx, other);
-      }
+      // Row max over both halves (lanes t and t ^ 16 hold one row).
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const float m_old = m_ref;
       if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
       const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
@@ -422,23 +412,23 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
 #pragma unroll 1
         for (int q = 0; q < DH / 32; ++q) {
           uint32_t ov[32];
-          tmem_ld32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
+          tmem_ld_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
+          tmem_st_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
         }
       }
       tc_fence_after();
       // P half row (bf16 pairs) -> TMEM P_b, the A operand of O += P V.
 #pragma unroll
-      for (int q = 0; q < HALF / 64; ++q)
-        tmem_st32(tmem + lane_off + C::TM_P + 64 * b + hf * (HALF / 2) + q * 32,
-                  *reinterpret_cast<const uint32_t(*)[32]>(pk + q * 32));
-      if constexpr (HALF % 64 != 0) {
+      if constexpr (HALF == 64) {
+        tmem_st_16x2_32<HALF / 2>(tmem + lane_off + C::TM_P + 64 * b,
+                                  *reinterpret_cast<const uint32_t(*)[32]>(pk));
+      } else {
         // BN = 64: a half row is 32 keys = 16 columns
-        tmem_st16(tmem + lane_off + C::TM_P + 64 * b + hf * (HALF / 2),
-                  *reinterpret_cast<const uint32_t(*)[16]>(pk));
+        tmem_st_16x2_16<HALF / 2>(tmem + lane_off + C::TM_P + 64 * b,
+                                  *reinterpret_cast<const uint32_t(*)[16]>(pk));
       }
       tmem_wait_st();
       tc_fence_before();
@@ -454,14 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       else tc_fence_after();
     }
     if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 3); }
-    // Row sum over both halves (exchange number n, after the n row-max exchanges).
-    float l_row = l;
-    if (ok && n > 0) {
-      bool good;
-      const float other = pair_exchange(n, l, good);
-      if (!good) { ok = false; *abort_flag = 1; report_fault(p.err, 5, 4); }
-      l_row += other;
-    }
+    // Row sum over both halves.
+    const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
     const int64_t grow = int64_t(i) * BN + row;           // row within the plane
     const bool store = row < BN && grow < p.n_pad;
     const bool have = ok && n > 0 && l_row > 0.f;
@@ -471,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     for (int q = 0; q < DH / 32; ++q) {
       uint32_t ov[32];
       if (ok && n > 0) {
-        tmem_ld32(tmem + lane_off + C::TM_O + hf * DH + q * 32, ov);
+        tmem_ld_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
         tmem_wait_ld();
       }
       uint32_t w[16];
