@@ -326,10 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       if (lane == 0) mbar_arrive(bar_s_free(b));
       if (tr) LVA_TRACE_AT(3, t);
 
-      // Real keys of this half (only the block holding the sequence end is partial).
+      // Real keys of this half (only the block holding the sequence end is partial).  The
+      // choice of path is made for the whole warp: the exponential loop below issues
+      // warp-collective TMEM stores, and the two halves of a row can differ at the end.
       const int64_t valid = p.n_valid - int64_t(j) * BN - hf * HALF;
+      const bool full = __all_sync(0xffffffffu, valid >= HALF);
       float mx;
-      if (valid >= HALF) {
+      if (full) {
         // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (3-input max, 4 chains)
         float m4[4];
         if (c >= 0.f) {
@@ -359,11 +362,20 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
       const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // P_b was last read by O += P(t-2) V; wait for it before any part of P(t) is stored.
+      // Each P buffer has its own completion barrier, so the wait never aliases an older
+      // phase.  (Almost always complete by now: P(t-2) V was issued a block earlier.)
+      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), ((t >> 1) - 1) & 1, abort_flag))) {
+        ok = false; break;
+      }
+      tc_fence_after();
+      const uint32_t p_tm = tmem + lane_off + C::TM_P + 64 * b;
       float r4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[HALF / 2];
-      if (valid >= HALF) {
+      if (full) {
         // Pairs of elements with packed fp32 math; every third pair takes its exponentials
-        // on the FMA pipe, the rest on the MUFU, which balances the two units.
+        // on the FMA pipe, the rest on the MUFU, which balances the two units.  With 64-key
+        // halves the first 16 pairs go to TMEM while the rest are computed.
         const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
         uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
@@ -381,6 +393,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           float p0, p1;
           f2_unpack(p2, p0, p1);
           pk[e] = pack_bf16x2(p0, p1);
+          if constexpr (HALF == 64) {
+            if (e == 15) tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          }
+        }
+        if constexpr (HALF == 64) {
+          tmem_st_16x2_16<HALF / 2>(p_tm + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
+        } else {
+          tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
         }
         float a0, a1, b0, b1;
         f2_unpack(acc[0], a0, a1);
@@ -394,15 +414,18 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           r4[(e >> 1) & 3] += p0 + p1;
           pk[e / 2] = pack_bf16x2(p0, p1);
         }
+        // P half row (bf16 pairs) -> TMEM P_b, the A operand of O += P V.
+        if constexpr (HALF == 64) {
+          tmem_st_16x2_32<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+        } else {
+          tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+        }
       }
       l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
       if (tr) LVA_TRACE_AT(4, t);
 
-      // P_b was last read by O += P(t-2) V; O itself by O += P(t-1) V.  Each P buffer has
-      // its own completion barrier, so these waits never alias an older phase.
-      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), ((t >> 1) - 1) & 1, abort_flag))) {
-        ok = false; break;
-      }
+      // O was last written by O += P(t-1) V: rescale it (rarely) once that has completed,
+      // before P(t) is released to the P V issuer.
       if (t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
         if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(b ^ 1), ((t - 1) >> 1) & 1, abort_flag))) {
           ok = false; break;
@@ -418,17 +441,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
           tmem_st_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
         }
-      }
-      tc_fence_after();
-      // P half row (bf16 pairs) -> TMEM P_b, the A operand of O += P V.
-#pragma unroll
-      if constexpr (HALF == 64) {
-        tmem_st_16x2_32<HALF / 2>(tmem + lane_off + C::TM_P + 64 * b,
-                                  *reinterpret_cast<const uint32_t(*)[32]>(pk));
-      } else {
-        // BN = 64: a half row is 32 keys = 16 columns
-        tmem_st_16x2_16<HALF / 2>(tmem + lane_off + C::TM_P + 64 * b,
-                                  *reinterpret_cast<const uint32_t(*)[16]>(pk));
       }
       tmem_wait_st();
       tc_fence_before();
