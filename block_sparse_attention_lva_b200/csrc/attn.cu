@@ -373,16 +373,17 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       float r4[4] = {0.f, 0.f, 0.f, 0.f};
       uint32_t pk[HALF / 2];
       if (full) {
-        // Pairs of elements with packed fp32 math; every third pair takes its exponentials
-        // on the FMA pipe, the rest on the MUFU, which balances the two units.  With 64-key
-        // halves the first 16 pairs go to TMEM while the rest are computed.
+        // Pairs of elements with packed fp32 math; every fourth pair takes its exponentials
+        // on the FMA pipe, the rest on the MUFU (of 1/2, 1/3, 1/4 and none on the FMA pipe,
+        // 1/4 measured fastest).  With 64-key halves the first 16 pairs go to TMEM while the
+        // rest are computed.
         const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
         uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
         for (int e = 0; e < HALF / 2; ++e) {
           const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
           uint64_t p2;
-          if (e % 3 == 2) {
+          if (e % 4 == 3) {
             p2 = exp2_poly_f2(x2);
           } else {
             float x0, x1;
