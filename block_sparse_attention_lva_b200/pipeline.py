@@ -94,8 +94,15 @@ class VideoBlockSparseAttention:
 
     @staticmethod
     def _stacked(q, k, v):
-        """True when q, k, v are consecutive, equally sized, contiguous slices of one buffer."""
+        """True when q, k, v are consecutive, equally sized, contiguous slices of one buffer.
+
+        Adjacent addresses are not enough: three separate allocations can sit back to back,
+        and a view spanning them would leave the first tensor's storage.
+        """
         if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+            return False
+        sq = q.untyped_storage()
+        if not (sq.data_ptr() == k.untyped_storage().data_ptr() == v.untyped_storage().data_ptr()):
             return False
         nbytes = q.numel() * q.element_size()
         return (k.data_ptr() == q.data_ptr() + nbytes and v.data_ptr() == k.data_ptr() + nbytes
@@ -133,6 +140,80 @@ class VideoBlockSparseAttention:
         self.attend()
         self.reorder_out()
         return self.o, self.lse
+
+
+    def forward_host(self, qkv_host, o_host, lse_host, step: int = 0, chunks: int = 6):
+        """One layer step from and to pinned host memory, with the copies overlapped.
+
+        ``qkv_host``: pinned bf16 [3, B, H, N, d] (raster Q, K, V); ``o_host``: pinned bf16
+        [B, H, N, d] (raster O, written); ``lse_host``: pinned fp32 [B, H, n_pad] (tile-order
+        LSE, written).  Heads are independent given the mask, so the step runs per group of
+        heads of one batch element: the host-to-device copy of group c+1 and the
+        device-to-host copy of group c-1 proceed while group c is reordered and attended.
+        Copies use their own streams; the call returns with the caller's current stream
+        ordered after the last copy back (synchronise that stream before reading o_host).
+        """
+        B, H, N, d = self.B, self.H, self.n_valid, self.d
+        assert tuple(qkv_host.shape) == (3, B, H, N, d) and qkv_host.is_pinned()
+        assert tuple(o_host.shape) == (B, H, N, d) and o_host.is_pinned()
+        assert tuple(lse_host.shape) == (B, H, self.n_pad) and lse_host.is_pinned()
+        if not hasattr(self, "_host_io"):
+            self._host_io = dict(
+                qkv_dev=torch.empty((3, B, H, N, d), dtype=torch.bfloat16, device=self.device),
+                h2d=torch.cuda.Stream(self.device), d2h=torch.cuda.Stream(self.device))
+        io = self._host_io
+        qkv_dev, s_h2d, s_d2h = io["qkv_dev"], io["h2d"], io["d2h"]
+        cur = torch.cuda.current_stream(self.device)
+        groups = []
+        per = max(1, -(-H // max(1, chunks // max(1, B))))
+        for b in range(B):
+            for h0 in range(0, H, per):
+                groups.append((b, h0, min(H, h0 + per)))
+        # Ordering: copies into the staging buffer wait for the previous step's compute.
+        s_h2d.wait_stream(cur)
+        s_d2h.wait_stream(cur)
+        self.build_mask(step)
+        in_ready, out_ready = [], []
+        for b, h0, h1 in groups:
+            with torch.cuda.stream(s_h2d):
+                for t in range(3):
+                    qkv_dev[t, b, h0:h1].copy_(qkv_host[t, b, h0:h1], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(s_h2d)
+            in_ready.append(ev)
+        # The static-mask and repetitive-head tables are indexed per head of the group.
+        nb = self.nb
+        for (b, h0, h1), ev in zip(groups, in_ready):
+            cur.wait_event(ev)
+            hn = h1 - h0
+            P = hn
+            for t, dst in ((0, self.q_t), (1, self.k_t), (2, self.v_t)):
+                lb.lva_reorder_tokens(qkv_dev[t, b, h0:h1].reshape(P, N, d),
+                                      dst[b, h0:h1].reshape(P, self.n_pad, d), self.grid, self.tile,
+                                      self.n_pad, inverse=False)
+            mh = self.mask_heads
+            row_ptr = self.row_ptr if mh == 1 else self.row_ptr[h0 * nb:]
+            qs = None
+            if self.query_src is not None:
+                qs = self.query_src if self.query_src.shape[0] == 1 else self.query_src[h0:h1]
+            lb.lva_block_sparse_attn(self.q_t[b:b + 1, h0:h1], self.k_t[b:b + 1, h0:h1],
+                                     self.v_t[b:b + 1, h0:h1], self.o_t[b:b + 1, h0:h1],
+                                     self.lse[b:b + 1, h0:h1], N, self.block_size, row_ptr, self.col_idx,
+                                     1 if mh == 1 else hn, self.scale, qs)
+            if qs is not None:
+                lb.lva_broadcast_blocks(self.o_t[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], self.block_size, qs)
+            lb.lva_reorder_tokens(self.o_t[b, h0:h1].reshape(P, self.n_pad, d), self.o[b, h0:h1].reshape(P, N, d),
+                                  self.grid, self.tile, self.n_pad, inverse=True)
+            ev = torch.cuda.Event()
+            ev.record(cur)
+            out_ready.append(ev)
+        for (b, h0, h1), ev in zip(groups, out_ready):
+            s_d2h.wait_event(ev)
+            with torch.cuda.stream(s_d2h):
+                o_host[b, h0:h1].copy_(self.o[b, h0:h1], non_blocking=True)
+                lse_host[b, h0:h1].copy_(self.lse[b, h0:h1], non_blocking=True)
+        cur.wait_stream(s_d2h)
+        return o_host, lse_host
 
 
 class SquadTwoPass:
