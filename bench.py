@@ -62,7 +62,7 @@ def _config_dict(w: Workload, spec: dict, n_gpus: int) -> dict:
                         f"{w.block_size}x{w.block_size} blocks, +-1 latent-frame window + 4 rotating "
                         f"anchor blocks, denoising step = step index mod 50",
             "global_batch": n_gpus * w.B, "heads": w.H, "head_dim": w.d, "seq_len": w.n_pad,
-            "block": w.block_size, "step_contents": "reorder of stacked QKV + CSR build (3 launches) + attention + inverse reorder",
+            "block": w.block_size, "step_contents": "reorder of stacked QKV + CSR build (3 launches) + attention with the inverse reorder fused into its epilogue",
             "l2": "inputs larger than L2 (302 MB Q/K/V per GPU), no flush",
             "parallelism": f"dp{n_gpus} (independent batch elements)"}
 
@@ -189,10 +189,9 @@ def run_lva(args):
         layer.build_mask(s)
         if ev is not None:
             ev[0].record(stream)
-        layer.attend()
+        layer.attend_to_raster()       # attention with the inverse reorder fused in
         if ev is not None:
             ev[1].record(stream)
-        layer.reorder_out()
 
     def barrier():
         if ws > 1:
@@ -275,7 +274,7 @@ def run_lva(args):
             "e2e": {"value": flops_all / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": ms_e2e / args.steps},
-            "gpu_launches": 6 * args.steps,
+            "gpu_launches": 5 * args.steps,
         }
         if ws == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, spec, args.cpu_seconds)

@@ -8,7 +8,8 @@ and fails if the library has not been built.
 from ._binding import (LVA_MASK_ALL, LVA_MASK_LVSA_FRAMES, LVA_MASK_STATIC, LVA_MASK_TWO_STAGE,
                        LVA_MASK_WINDOW_ANCHOR,
                        LIB_PATH, LvaError, MaskParams, lva_block_mask_max_nnz, lva_block_sparse_attn,
-                       lva_aggregate_masks, lva_block_energy, lva_broadcast_blocks,
+                       lva_aggregate_masks, lva_block_energy, lva_block_sparse_attn_raster,
+                       lva_broadcast_blocks,
                        lva_build_block_mask, lva_device_error, lva_reorder_tokens, lva_select_blocks,
                        lva_version)
 from .pipeline import SquadTwoPass, StaticMaskCalibrator, VideoBlockSparseAttention, mask_params_for
@@ -16,5 +17,5 @@ from .pipeline import SquadTwoPass, StaticMaskCalibrator, VideoBlockSparseAttent
 __all__ = ["LVA_MASK_ALL", "LVA_MASK_LVSA_FRAMES", "LVA_MASK_STATIC", "LVA_MASK_TWO_STAGE", "LVA_MASK_WINDOW_ANCHOR", "LIB_PATH",
            "LvaError", "MaskParams", "lva_block_mask_max_nnz", "lva_block_sparse_attn", "lva_broadcast_blocks",
            "lva_build_block_mask", "lva_device_error", "lva_reorder_tokens", "lva_version",
-           "lva_block_energy", "lva_select_blocks", "lva_aggregate_masks",
+           "lva_block_energy", "lva_select_blocks", "lva_aggregate_masks", "lva_block_sparse_attn_raster",
            "SquadTwoPass", "StaticMaskCalibrator", "VideoBlockSparseAttention", "mask_params_for"]

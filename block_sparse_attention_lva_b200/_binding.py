@@ -47,6 +47,9 @@ SIGNATURES = {
     "lva_build_block_mask": (_c_int, [ctypes.POINTER(LvaMaskParams), _vp, _vp, _vp, _c_i64, _vp, _vp]),
     "lva_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
                                        _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp, _c_int, _vp]),
+    "lva_block_sparse_attn_raster": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
+                                              _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _c_int, _c_int,
+                                              _c_int, _c_int, _c_int, _c_int, _vp]),
     "lva_broadcast_blocks": (_c_int, [_vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _vp, _c_int, _vp]),
     "lva_block_energy": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int, _c_int,
                                   _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp]),
@@ -202,6 +205,29 @@ def lva_block_sparse_attn(q, k, v, o, lse, n_valid: int, block_size: int, row_pt
                                      mask_heads, ctypes.c_float(scale), _ptr(query_src), src_heads,
                                      ctypes.c_void_p(_stream(q.device))))
     return o, lse
+
+
+def lva_block_sparse_attn_raster(q, k, v, o_raster, lse, n_valid: int, block_size: int, row_ptr, col_idx,
+                                 mask_heads: int, scale: float, grid, tile):
+    """Block-sparse attention on tile-order Q, K, V with O written in raster order
+    ([B, H, n_valid, d]); LSE stays in tile order ([B, H, n_pad])."""
+    import torch
+    B, H, n_pad, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _cuda_tensor(t, name, torch.bfloat16)
+        _need(tuple(t.shape) == (B, H, n_pad, d), f"{name} must have shape {(B, H, n_pad, d)}")
+    _cuda_tensor(o_raster, "o_raster", torch.bfloat16, B * H * n_valid * d)
+    _cuda_tensor(lse, "lse", torch.float32, B * H * n_pad)
+    nb = n_pad // block_size
+    _cuda_tensor(row_ptr, "row_ptr", torch.int32, mask_heads * nb + 1)
+    _cuda_tensor(col_idx, "col_idx", torch.int32)
+    T, Hg, Wg = grid
+    tt, th, tw = tile
+    _check(lib.lva_block_sparse_attn_raster(_ptr(q), _ptr(k), _ptr(v), _ptr(o_raster), _ptr(lse), B, H, n_pad,
+                                            n_valid, d, block_size, _ptr(row_ptr), _ptr(col_idx),
+                                            col_idx.numel(), mask_heads, ctypes.c_float(scale), T, Hg, Wg,
+                                            tt, th, tw, ctypes.c_void_p(_stream(q.device))))
+    return o_raster, lse
 
 
 def lva_broadcast_blocks(o, lse, block_size: int, query_src):

@@ -175,39 +175,71 @@ lva_status lva_build_block_mask(const lva_mask_params* p, const uint8_t* dense_m
   return from_cuda(launch_build_mask(a, stream), "mask launch");
 }
 
+static lva_status attn_common(const char* fn, const void* q, const void* k, const void* v, void* o,
+                              float* lse, int B, int H, int64_t n_pad, int64_t n_valid, int d,
+                              int block_size, const int32_t* row_ptr, const int32_t* col_idx,
+                              int64_t col_len, int mask_heads, float scale, const int32_t* query_src,
+                              int src_heads, void* o_raster, int T, int Hg, int Wg, int tile_t,
+                              int tile_h, int tile_w, cudaStream_t stream) {
+  if (B < 0 || H < 1) return fail(LVA_ERR_INVALID_ARG, "%s: need B >= 0 and H >= 1", fn);
+  if (d != 64 && d != 128) return fail(LVA_ERR_UNSUPPORTED, "%s: head dim must be 64 or 128", fn);
+  if (block_size != 64 && block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "%s: block_size must be 64 or 128", fn);
+  if (n_pad <= 0 || n_pad % block_size != 0) return fail(LVA_ERR_INVALID_ARG, "%s: n_pad must be a positive multiple of block_size", fn);
+  if (n_valid < 0 || n_valid > n_pad) return fail(LVA_ERR_INVALID_ARG, "%s: need 0 <= n_valid <= n_pad", fn);
+  if (mask_heads != 1 && mask_heads != H) return fail(LVA_ERR_INVALID_ARG, "%s: mask_heads must be 1 or H", fn);
+  if (int64_t(B) * H * n_pad >= (int64_t(1) << 31)) return fail(LVA_ERR_UNSUPPORTED, "%s: B*H*n_pad must be < 2^31", fn);
+  if (!(scale == scale)) return fail(LVA_ERR_INVALID_ARG, "%s: scale is NaN", fn);
+  if (col_len < 0) return fail(LVA_ERR_INVALID_ARG, "%s: col_len < 0", fn);
+  if (query_src != nullptr && src_heads != 1 && src_heads != H)
+    return fail(LVA_ERR_INVALID_ARG, "%s: src_heads must be 1 or H", fn);
+  if (query_src != nullptr && !aligned(query_src, 4))
+    return fail(LVA_ERR_INVALID_ARG, "%s: query_src must be 4-byte aligned", fn);
+  if (o_raster != nullptr) {
+    if (T < 1 || Hg < 1 || Wg < 1 || tile_t < 1 || tile_h < 1 || tile_w < 1)
+      return fail(LVA_ERR_INVALID_ARG, "%s: grid and tile extents must be >= 1", fn);
+    if (int64_t(T) * Hg * Wg != n_valid)
+      return fail(LVA_ERR_INVALID_ARG, "%s: T*H*W must equal n_valid", fn);
+  }
+  if (B == 0) return ok();
+  if (!q || !k || !v || !(o || o_raster) || !lse || !row_ptr || (!col_idx && col_len > 0))
+    return fail(LVA_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || (o && !aligned(o, 16)) ||
+      (o_raster && !aligned(o_raster, 16)))
+    return fail(LVA_ERR_INVALID_ARG, "%s: q, k, v, o must be 16-byte aligned", fn);
+  if (!aligned(lse, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4))
+    return fail(LVA_ERR_INVALID_ARG, "%s: lse, row_ptr, col_idx must be 4-byte aligned", fn);
+  int* err = device_error_word();
+  if (err == nullptr) return fail(LVA_ERR_CUDA, "%s: cannot locate the device error word", fn);
+  AttnArgs a{q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr,
+             col_idx, col_len, mask_heads, scale, query_src, src_heads, err,
+             o_raster, T, Hg, Wg, tile_t, tile_h, tile_w};
+  const char* why = "launch";
+  cudaError_t e = launch_attn(a, stream, &why);
+  if (e != cudaSuccess) return fail(LVA_ERR_CUDA, "%s: %s: %s", fn, why, cudaGetErrorString(e));
+  return ok();
+}
+
 lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, void* o, float* lse,
                                  int B, int H, int64_t n_pad, int64_t n_valid, int d, int block_size,
                                  const int32_t* row_ptr, const int32_t* col_idx, int64_t col_len,
                                  int mask_heads, float scale, const int32_t* query_src, int src_heads,
                                  cudaStream_t stream) {
-  if (B < 0 || H < 1) return fail(LVA_ERR_INVALID_ARG, "attn: need B >= 0 and H >= 1");
-  if (d != 64 && d != 128) return fail(LVA_ERR_UNSUPPORTED, "attn: head dim must be 64 or 128");
-  if (block_size != 64 && block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "attn: block_size must be 64 or 128");
-  if (n_pad <= 0 || n_pad % block_size != 0) return fail(LVA_ERR_INVALID_ARG, "attn: n_pad must be a positive multiple of block_size");
-  if (n_valid < 0 || n_valid > n_pad) return fail(LVA_ERR_INVALID_ARG, "attn: need 0 <= n_valid <= n_pad");
-  if (mask_heads != 1 && mask_heads != H) return fail(LVA_ERR_INVALID_ARG, "attn: mask_heads must be 1 or H");
-  if (int64_t(B) * H * n_pad >= (int64_t(1) << 31)) return fail(LVA_ERR_UNSUPPORTED, "attn: B*H*n_pad must be < 2^31");
-  if (!(scale == scale)) return fail(LVA_ERR_INVALID_ARG, "attn: scale is NaN");
-  if (col_len < 0) return fail(LVA_ERR_INVALID_ARG, "attn: col_len < 0");
-  if (query_src != nullptr && src_heads != 1 && src_heads != H)
-    return fail(LVA_ERR_INVALID_ARG, "attn: src_heads must be 1 or H");
-  if (query_src != nullptr && !aligned(query_src, 4))
-    return fail(LVA_ERR_INVALID_ARG, "attn: query_src must be 4-byte aligned");
-  if (B == 0) return ok();
-  if (!q || !k || !v || !o || !lse || !row_ptr || (!col_idx && col_len > 0))
-    return fail(LVA_ERR_INVALID_ARG, "attn: null pointer");
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
-    return fail(LVA_ERR_INVALID_ARG, "attn: q, k, v, o must be 16-byte aligned");
-  if (!aligned(lse, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4))
-    return fail(LVA_ERR_INVALID_ARG, "attn: lse, row_ptr, col_idx must be 4-byte aligned");
-  int* err = device_error_word();
-  if (err == nullptr) return fail(LVA_ERR_CUDA, "attn: cannot locate the device error word");
-  AttnArgs a{q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr,
-             col_idx, col_len, mask_heads, scale, query_src, src_heads, err};
-  const char* why = "launch";
-  cudaError_t e = launch_attn(a, stream, &why);
-  if (e != cudaSuccess) return fail(LVA_ERR_CUDA, "attn: %s: %s", why, cudaGetErrorString(e));
-  return ok();
+  if (o == nullptr && B > 0) return fail(LVA_ERR_INVALID_ARG, "attn: null pointer");
+  return attn_common("attn", q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr, col_idx,
+                     col_len, mask_heads, scale, query_src, src_heads, nullptr, 0, 0, 0, 0, 0, 0,
+                     stream);
+}
+
+lva_status lva_block_sparse_attn_raster(const void* q, const void* k, const void* v, void* o_raster,
+                                        float* lse, int B, int H, int64_t n_pad, int64_t n_valid,
+                                        int d, int block_size, const int32_t* row_ptr,
+                                        const int32_t* col_idx, int64_t col_len, int mask_heads,
+                                        float scale, int T, int Hg, int Wg, int tile_t, int tile_h,
+                                        int tile_w, cudaStream_t stream) {
+  if (o_raster == nullptr && B > 0) return fail(LVA_ERR_INVALID_ARG, "attn_raster: null pointer");
+  return attn_common("attn_raster", q, k, v, nullptr, lse, B, H, n_pad, n_valid, d, block_size,
+                     row_ptr, col_idx, col_len, mask_heads, scale, nullptr, 1, o_raster, T, Hg, Wg,
+                     tile_t, tile_h, tile_w, stream);
 }
 
 lva_status lva_broadcast_blocks(void* o, float* lse, int B, int H, int64_t n_pad, int d, int block_size,

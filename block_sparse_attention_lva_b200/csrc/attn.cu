@@ -31,6 +31,7 @@
 
 #include "kernels.h"
 #include "ptx.cuh"
+#include "tile_order.cuh"
 
 namespace lva {
 namespace {
@@ -65,7 +66,9 @@ struct AttnParams {
   const int32_t* row_ptr;
   const int32_t* col_idx;
   int64_t col_len;
-  __nv_bfloat16* o;
+  __nv_bfloat16* o;                // tile order [planes, n_pad, D], or
+  __nv_bfloat16* o_raster;         // when set: raster order [planes, n_valid, D] (o unused)
+  Grid3 grid;                      // latent grid and tile of the raster order
   float* lse;
   const int32_t* query_src;        // NULL or [src_heads, nb]: blocks copied from an anchor
   int src_heads;
@@ -463,7 +466,17 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     const bool store = row < BN && grow < p.n_pad;
     const bool have = ok && n > 0 && l_row > 0.f;
     const float inv_l = have ? 1.f / l_row : 0.f;
-    __nv_bfloat16* orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
+    // O row destination: tile order, or (fused inverse reorder) the row's raster position;
+    // padding rows have no raster position and are not written then.
+    __nv_bfloat16* orow;
+    bool store_o = store;
+    if (p.o_raster != nullptr) {
+      store_o = store && grow < p.n_valid;
+      const uint32_t raster = store_o ? tile_order_to_raster(uint32_t(grow), p.grid) : 0u;
+      orow = p.o_raster + (plane * p.n_valid + int64_t(raster)) * D + hf * DH;
+    } else {
+      orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
+    }
 #pragma unroll 1
     for (int q = 0; q < DH / 32; ++q) {
       uint32_t ov[32];
@@ -475,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
 #pragma unroll
       for (int e = 0; e < 16; ++e)
         w[e] = have ? pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l) : 0u;
-      if (store) {
+      if (store_o) {
         uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
 #pragma unroll
         for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
@@ -554,6 +567,9 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   p.col_idx = a.col_idx;
   p.col_len = a.col_len;
   p.o = static_cast<__nv_bfloat16*>(a.o);
+  p.o_raster = static_cast<__nv_bfloat16*>(a.o_raster);
+  p.grid = Grid3{uint32_t(a.T), uint32_t(a.Hg), uint32_t(a.Wg), uint32_t(a.tt), uint32_t(a.th),
+                 uint32_t(a.tw)};
   p.lse = a.lse;
   p.query_src = a.query_src;
   p.src_heads = a.src_heads;

@@ -51,6 +51,8 @@ struct AttnArgs {
   const int32_t* query_src;  // NULL or [src_heads, nb]
   int src_heads;
   int* err;  // device error word
+  void* o_raster;            // NULL, or O in raster order [B, H, n_valid, d] instead of o
+  int T, Hg, Wg, tt, th, tw; // latent grid and tile (used with o_raster)
 };
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why);
 

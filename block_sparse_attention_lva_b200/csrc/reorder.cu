@@ -10,36 +10,10 @@
 #include <cstdint>
 
 #include "kernels.h"
+#include "tile_order.cuh"
 
 namespace lva {
 namespace {
-
-struct Grid3 {
-  uint32_t T, H, W, tt, th, tw;
-};
-
-// Raster index of the k-th token in tile order (k < T*H*W).
-__device__ __forceinline__ uint32_t tile_order_to_raster(uint32_t k, const Grid3& g) {
-  const uint32_t hw = g.H * g.W;
-  const uint32_t slab = g.tt * hw;                 // tokens in a full depth-tt slab
-  const uint32_t it = k / slab;
-  uint32_t r = k - it * slab;
-  const uint32_t dt = min(g.tt, g.T - it * g.tt);  // depth of this slab (last may be short)
-  const uint32_t row_tokens = dt * g.th * g.W;     // tokens in a full-height tile row
-  const uint32_t ih = r / row_tokens;
-  r -= ih * row_tokens;
-  const uint32_t dh = min(g.th, g.H - ih * g.th);
-  const uint32_t tile_tokens = dt * dh * g.tw;     // tokens in a full-width tile of this row
-  const uint32_t iw = r / tile_tokens;
-  r -= iw * tile_tokens;
-  const uint32_t dw = min(g.tw, g.W - iw * g.tw);
-  const uint32_t plane = dh * dw;
-  const uint32_t t1 = r / plane;
-  r -= t1 * plane;
-  const uint32_t h1 = r / dw;
-  const uint32_t w1 = r - h1 * dw;
-  return (it * g.tt + t1) * hw + (ih * g.th + h1) * g.W + (iw * g.tw + w1);
-}
 
 template <int CHUNK>
 struct Vec;

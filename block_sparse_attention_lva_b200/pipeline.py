@@ -8,6 +8,9 @@ once through torch, which is used only for device memory and streams) and runs, 
    change with the step; static, two-stage and all-ones masks are built once);
 3. ``lva_block_sparse_attn`` -> O (tile order) and LSE;
 4. ``lva_reorder_tokens`` inverse on O (tile order -> raster [B, H, N, d]).
+
+Steps 3 and 4 run as one launch (``lva_block_sparse_attn_raster``) unless repetitive heads
+need the tile-order broadcast between them.
 """
 from __future__ import annotations
 
@@ -127,6 +130,13 @@ class VideoBlockSparseAttention:
         if self.query_src is not None:
             lb.lva_broadcast_blocks(self.o_t, self.lse, self.block_size, self.query_src)
 
+    def attend_to_raster(self):
+        """Attention with the inverse reorder fused into its epilogue: O goes straight to
+        raster order (``self.o``); LSE stays in tile order (``self.lse``)."""
+        lb.lva_block_sparse_attn_raster(self.q_t, self.k_t, self.v_t, self.o, self.lse, self.n_valid,
+                                        self.block_size, self.row_ptr, self.col_idx, self.mask_heads,
+                                        self.scale, self.grid, self.tile)
+
     def reorder_out(self):
         P = self.B * self.H
         lb.lva_reorder_tokens(self.o_t.view(P, self.n_pad, self.d), self.o.view(P, self.n_valid, self.d),
@@ -137,8 +147,11 @@ class VideoBlockSparseAttention:
         buffer ``self.o``) and tile-order LSE ``self.lse``."""
         self.reorder_in(q, k, v)
         self.build_mask(step)
-        self.attend()
-        self.reorder_out()
+        if self.query_src is None:
+            self.attend_to_raster()        # steps 3 and 4 in one launch
+        else:
+            self.attend()                  # repetitive heads broadcast in tile order
+            self.reorder_out()
         return self.o, self.lse
 
 
@@ -193,17 +206,20 @@ class VideoBlockSparseAttention:
                                       self.n_pad, inverse=False)
             mh = self.mask_heads
             row_ptr = self.row_ptr if mh == 1 else self.row_ptr[h0 * nb:]
-            qs = None
-            if self.query_src is not None:
+            qkv_t = (self.q_t[b:b + 1, h0:h1], self.k_t[b:b + 1, h0:h1], self.v_t[b:b + 1, h0:h1])
+            if self.query_src is None:
+                lb.lva_block_sparse_attn_raster(*qkv_t, self.o[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], N,
+                                                self.block_size, row_ptr, self.col_idx, 1 if mh == 1 else hn,
+                                                self.scale, self.grid, self.tile)
+            else:
                 qs = self.query_src if self.query_src.shape[0] == 1 else self.query_src[h0:h1]
-            lb.lva_block_sparse_attn(self.q_t[b:b + 1, h0:h1], self.k_t[b:b + 1, h0:h1],
-                                     self.v_t[b:b + 1, h0:h1], self.o_t[b:b + 1, h0:h1],
-                                     self.lse[b:b + 1, h0:h1], N, self.block_size, row_ptr, self.col_idx,
-                                     1 if mh == 1 else hn, self.scale, qs)
-            if qs is not None:
+                lb.lva_block_sparse_attn(*qkv_t, self.o_t[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], N,
+                                         self.block_size, row_ptr, self.col_idx, 1 if mh == 1 else hn,
+                                         self.scale, qs)
                 lb.lva_broadcast_blocks(self.o_t[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], self.block_size, qs)
-            lb.lva_reorder_tokens(self.o_t[b, h0:h1].reshape(P, self.n_pad, d), self.o[b, h0:h1].reshape(P, N, d),
-                                  self.grid, self.tile, self.n_pad, inverse=True)
+                lb.lva_reorder_tokens(self.o_t[b, h0:h1].reshape(P, self.n_pad, d),
+                                      self.o[b, h0:h1].reshape(P, N, d), self.grid, self.tile, self.n_pad,
+                                      inverse=True)
             ev = torch.cuda.Event()
             ev.record(cur)
             out_ready.append(ev)

@@ -181,6 +181,30 @@ lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, vo
                                  const int32_t* query_src, int src_heads, cudaStream_t stream);
 
 /*
+ * lva_block_sparse_attn_raster -- lva_block_sparse_attn with O written in raster order.
+ *
+ * The same attention as lva_block_sparse_attn on tile-order q, k, v (same definition, same
+ * arithmetic, same LSE in tile order), with the inverse token reorder fused into the output:
+ * the row at tile-order position r < n_valid of plane p is stored at its raster position,
+ *   o_raster[p][raster(r)][:]   with raster() the tile order of lva_reorder_tokens for the
+ *                               grid T x Hg x Wg and tiles tile_t x tile_h x tile_w,
+ * and padded rows (r >= n_valid) are not stored.  This is the attention and the inverse
+ * reorder of one layer (LVSA page, technical summary section 2; CalibAtt page, section 2 B)
+ * in one launch.
+ *
+ * o_raster: device bf16 [B, H, n_valid, d], 16-byte aligned (written).  Requires
+ * T*Hg*Wg == n_valid and extents >= 1.  Repetitive-head maps (query_src) are not accepted
+ * here: their broadcast works in tile order, so use lva_block_sparse_attn for them.  Other
+ * arguments, support and errors as for lva_block_sparse_attn.
+ */
+lva_status lva_block_sparse_attn_raster(const void* q, const void* k, const void* v, void* o_raster,
+                                        float* lse, int B, int H, int64_t n_pad, int64_t n_valid,
+                                        int d, int block_size, const int32_t* row_ptr,
+                                        const int32_t* col_idx, int64_t col_len, int mask_heads,
+                                        float scale, int T, int Hg, int Wg, int tile_t, int tile_h,
+                                        int tile_w, cudaStream_t stream);
+
+/*
  * lva_broadcast_blocks -- fill the query blocks of repetitive heads from their anchors.
  *
  * CalibAtt page ("Accelerating Text-to-Video Generation with Calibrated Sparse Attention",
