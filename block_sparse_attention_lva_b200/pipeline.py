@@ -243,6 +243,9 @@ class SquadTwoPass:
 
         O = T^-1( Attn_G( T(Q), T(K), T(Attn_L(Q, K, V)) ) )
 
+    (T^-1 is applied by the global pass's epilogue, which stores each row at its position in
+    the original order.)
+
     ``window`` and ``m`` must be multiples of ``block_size``; inputs are [B, H, n, d] bf16 in
     the order whose consecutive tokens form the windows (e.g. after the spatiotemporal tile
     reorder).
@@ -260,7 +263,6 @@ class SquadTwoPass:
         self.o_local = torch.empty(shape, dtype=torch.bfloat16, **kw)
         self.qk_t = torch.empty((2,) + shape, dtype=torch.bfloat16, **kw)     # transposed Q, K
         self.o_local_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
-        self.o_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
         self.o = torch.empty(shape, dtype=torch.bfloat16, **kw)
         self.lse_local = torch.empty((B, H, n), dtype=torch.float32, **kw)
         self.lse_global_t = torch.empty((B, H, n), dtype=torch.float32, **kw)
@@ -293,9 +295,9 @@ class SquadTwoPass:
             self._transpose(k, self.qk_t[1], P)
         self._transpose(self.o_local, self.o_local_t, P)
         rp, ci = self.csr["global"]
-        lb.lva_block_sparse_attn(self.qk_t[0], self.qk_t[1], self.o_local_t, self.o_t, self.lse_global_t,
-                                 self.n, self.block_size, rp, ci, 1, self.scale)
-        self._transpose(self.o_t, self.o, P, inverse=True)
+        # The inverse window transpose is the raster store of the global pass's epilogue.
+        lb.lva_block_sparse_attn_raster(self.qk_t[0], self.qk_t[1], self.o_local_t, self.o, self.lse_global_t,
+                                        self.n, self.block_size, rp, ci, 1, self.scale, self.grid, self.tile)
         return self.o
 
 
