@@ -306,6 +306,76 @@ def _oracle_sample(w, spec, q, k, v, perm, seconds, seed):
     return flops, time.perf_counter() - t0, items
 
 
+def _oracle_mask_for(w, spec, step=0):
+    """Dense block mask [H_m, nb, nb] of a mask specification, from the oracle."""
+    from oracle.mask import all_mask, lvsa_frame_mask, two_stage_mask, window_anchor_mask
+    from synthetic import static_calibrated_mask
+    kind = spec["kind"]
+    if kind == "window_anchor":
+        return window_anchor_mask(w.n_pad, w.n_valid, w.block_size, spec["unit"], spec["radius"],
+                                  spec["anchors"], step)[None]
+    if kind == "two_stage":
+        return two_stage_mask(w.nb, spec["group"])[None]
+    if kind == "all":
+        return all_mask(w.nb)[None]
+    if kind == "lvsa_frames":
+        return lvsa_frame_mask(w.n_pad, w.n_valid, w.block_size, spec["unit"], spec["anchors"], step,
+                               spec["budget"])[None]
+    if kind == "static":
+        return static_calibrated_mask(w, spec["density"]).astype(bool)
+    raise ValueError(kind)
+
+
+def run_oracle_report(args, gpu_ms):
+    """The FP64 oracle timed per (workload, mask) on a seeded sample of (head, query block)
+    items -- the first and last query block of every head, then random ones -- for about
+    ``args.cpu_seconds`` / 4 each, extrapolated to the whole launch by active block pairs."""
+    from oracle.attention import attention_blocked
+    from oracle.reorder import reorder_forward, tile_permutation
+    budget = max(2.0, args.cpu_seconds / 4)
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    for name in ("tiny", "small", "static", "large", "long"):
+        w = WORKLOADS[name]
+        q, k, v = make_qkv(w)
+        perm = tile_permutation(w.T, w.Hg, w.Wg, *w.tile)
+        P = w.B * w.H
+        tile = [torch.from_numpy(reorder_forward(x.view(torch.int16).reshape(P, w.n_valid, w.d).numpy(), perm,
+                                                 w.n_pad)).view(torch.bfloat16).reshape(w.B, w.H, w.n_pad, w.d)
+                for x in (q, k, v)]
+        for spec in mask_variants(w):
+            m = _oracle_mask_for(w, spec)
+            total_pairs = int(m.sum()) * (w.H if m.shape[0] == 1 else 1) * w.B
+            rng = np.random.default_rng(11)
+            order = [(h, 0) for h in range(w.H)] + [(h, w.nb - 1) for h in range(w.H)]
+            flops, items = 0.0, 0
+            t0 = time.perf_counter()
+            while (time.perf_counter() - t0 < budget or items < 4) and items < w.H * w.nb:
+                h, i = order[items] if items < len(order) else (int(rng.integers(0, w.H)), int(rng.integers(0, w.nb)))
+                hm = h if m.shape[0] > 1 else 0
+                attention_blocked(tile[0][:, h:h + 1], tile[1][:, h:h + 1], tile[2][:, h:h + 1], m[hm:hm + 1],
+                                  w.block_size, w.n_valid, w.scale, query_blocks=[(0, 0, i)])
+                flops += int(m[hm, i].sum()) * _flops_per_nnz(w)
+                items += 1
+            secs = time.perf_counter() - t0
+            rate = flops / secs
+            full_s = total_pairs * _flops_per_nnz(w) / rate
+            line = {"report": "oracle", "workload": name, "mask": spec["label"], "sample_items": items,
+                    "sample_s": secs, "oracle_tflops": rate / 1e12, "cores": _threads(), "cpu_model": model,
+                    "full_launch_s_extrapolated": full_s}
+            ms = gpu_ms.get((name, spec["label"]))
+            if ms:
+                line["gpu_attn_ms"] = ms
+                line["speedup_vs_oracle"] = full_s * 1e3 / ms
+            print(json.dumps(line), flush=True)
+
+
 def _threads():
     try:
         from threadpoolctl import threadpool_info
@@ -353,12 +423,16 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def _time_cuda(fn, reps=7, warmup=2):
-    """Median ms of `fn` over `reps` launches (CUDA events on the current stream)."""
+def _time_cuda(fn, reps=20, warmup=5, flush=None):
+    """Median ms of `fn` over `reps` launches (CUDA events on the current stream).  With
+    ``flush`` (a device buffer larger than L2), the buffer is rewritten before every timed
+    launch, outside the timed interval, so each launch starts with a cold L2."""
     for _ in range(warmup):
         fn()
     ts = []
     for _ in range(reps):
+        if flush is not None:
+            flush.add_(1)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         fn()
@@ -377,12 +451,16 @@ def run_report(args):
     dev = torch.device("cuda", 0)
     burst, sustained, hbm, peak_kind = _peaks()
     names = args.report.split(",")
+    l2_flush = torch.zeros(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MB > 126 MB L2
+    gpu_ms = {}
     for name in names:
-        if name in ("stress", "squad", "calib"):
+        if name in ("stress", "squad", "calib", "oracle"):
             continue
         w = WORKLOADS[name]
         q, k, v = make_qkv(w)
-        qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+        qkv_dev = torch.stack([q, k, v]).to(dev)
+        qkv_stacked = (qkv_dev[0], qkv_dev[1], qkv_dev[2])
+        qd, kd, vd = qkv_stacked
         del q, k, v
         sweep = []
         for spec in mask_variants(w):
@@ -395,6 +473,15 @@ def run_report(args):
             pairs = nnz * (w.B * w.H if layer.mask_heads == 1 else w.B)
             flops = pairs * _flops_per_nnz(w)
             ms = _time_cuda(layer.attend)
+            # roofline bound of this launch: tensor work at the sustained peak vs algorithmic
+            # bytes (Q, K, V read once, O written once, LSE) at the measured copy bandwidth
+            algo_bytes = w.B * w.H * (4 * w.n_pad * w.d * 2 + 4 * w.n_pad)
+            t_tensor, t_hbm = flops / (sustained * 1e9), algo_bytes / (hbm * 1e6)
+            bound_ms = max(t_tensor, t_hbm)
+            # the whole layer path: stacked reorder + CSR + attention with the fused inverse
+            ms_layer = _time_cuda(lambda: (layer.reorder_in(*qkv_stacked), setattr(layer, "_built_step", None),
+                                           layer.build_mask(0), layer.attend_to_raster()))
+            ms_flushed = _time_cuda(layer.attend, reps=10, flush=l2_flush) if name == "small" else None
             layer._built_step = None
             ms_mask = _time_cuda(lambda: (setattr(layer, "_built_step", None), layer.build_mask(0)))
             mask_bytes = (layer.mask_heads * w.nb * w.nb if spec["kind"] == "static" else 0) \
@@ -407,11 +494,17 @@ def run_report(args):
             line = {"report": name, "mask": spec["label"], "active_pairs": pairs,
                     "density": nnz / (layer.mask_heads * w.nb * w.nb), "attn_ms": ms,
                     "tflops": flops / ms / 1e9, "frac_of_sustained": flops / ms / 1e9 / sustained,
-                    "frac_of_burst": flops / ms / 1e9 / burst, "mask_build_us": ms_mask * 1e3,
+                    "frac_of_burst": flops / ms / 1e9 / burst,
+                    "bound": "tensor" if t_tensor >= t_hbm else "hbm", "bound_ms": bound_ms,
+                    "frac_of_bound": bound_ms / ms, "algorithmic_bytes": algo_bytes,
+                    "kv_l2_reread_bytes": pairs * 2 * w.block_size * w.d * 2,
+                    "layer_path_ms": ms_layer, "attn_ms_l2_flushed": ms_flushed,
+                    "mask_build_us": ms_mask * 1e3,
                     "mask_gbs": mask_bytes / ms_mask / 1e6, "reorder_ms": ms_reorder,
                     "reorder_gbs": reorder_bytes / ms_reorder / 1e6, "hbm_peak_gbs": hbm,
                     "peak_kind": peak_kind, "kernel_error": status}
             print(json.dumps(line), flush=True)
+            gpu_ms[(name, spec["label"])] = ms
             if spec["kind"] in ("window_anchor", "all"):
                 sweep.append((pairs, ms, nnz / (layer.mask_heads * w.nb * w.nb)))
             del layer
@@ -427,7 +520,7 @@ def run_report(args):
             print(json.dumps({"report": name, "density_sweep": [{"density": float(dd), "ms": float(m)} for _, m, dd in sweep],
                               "fit_ms": {"intercept": float(a), "per_pair_us": float(b * 1e3), "r2": float(r2),
                                          "intercept_share_of_10pct": float(a / y[i10])}}), flush=True)
-        del qd, kd, vd
+        del qd, kd, vd, qkv_dev, qkv_stacked
         torch.cuda.empty_cache()
     # SQuad's exact two-stage operator: 12 heads, 131,072 tokens (64 frames of 32 x 64),
     # windows of 512 tokens (m = 256 windows): local pass, window transpose, global pass.
@@ -500,6 +593,10 @@ def run_report(args):
         byts = hm * nb * nb + 4 * (hm * nb + 1) + 4 * n
         print(json.dumps({"report": "mask_stress", "mask_heads": hm, "nb": nb, "nnz": n, "ms": ms,
                           "gbs": byts / ms / 1e6, "hbm_peak_gbs": hbm}), flush=True)
+        del dense, col_idx
+        torch.cuda.empty_cache()
+    if "oracle" in names:
+        run_oracle_report(args, gpu_ms)
 
 
 def main():
@@ -511,7 +608,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--report", default="", help="comma list of workloads (tiny,small,static,large,long,stress,squad,calib): "
+    ap.add_argument("--report", default="", help="comma list of workloads (tiny,small,static,large,long,stress,squad,calib,oracle): "
                     "per-mask kernel timings and the density sweep fit instead of the bench line")
     ap.add_argument("--report-stress", action="store_true")
     args = ap.parse_args()
