@@ -50,6 +50,8 @@ SIGNATURES = {
     "lva_block_sparse_attn_raster": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
                                               _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _c_int, _c_int,
                                               _c_int, _c_int, _c_int, _c_int, _vp]),
+    "lva_window_transposed_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int,
+                                            _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp]),
     "lva_broadcast_blocks": (_c_int, [_vp, _vp, _c_int, _c_int, _c_i64, _c_int, _c_int, _vp, _c_int, _vp]),
     "lva_block_energy": (_c_int, [_vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int, _c_int,
                                   _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp]),
@@ -228,6 +230,25 @@ def lva_block_sparse_attn_raster(q, k, v, o_raster, lse, n_valid: int, block_siz
                                             col_idx.numel(), mask_heads, ctypes.c_float(scale), T, Hg, Wg,
                                             tt, th, tw, ctypes.c_void_p(_stream(q.device))))
     return o_raster, lse
+
+
+def lva_window_transposed_attn(q, k, v, o, lse, window: int, block_size: int, row_ptr, col_idx,
+                               mask_heads: int, scale: float):
+    """Block-sparse attention on the window-transposed order of q, k, v ([B, H, n, d], read in
+    place); O is stored in the input order, LSE ([B, H, n]) in the transposed order."""
+    import torch
+    B, H, n, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _cuda_tensor(t, name, torch.bfloat16)
+        _need(tuple(t.shape) == (B, H, n, d), f"{name} must have shape {(B, H, n, d)}")
+    _cuda_tensor(lse, "lse", torch.float32, B * H * n)
+    nb = n // block_size
+    _cuda_tensor(row_ptr, "row_ptr", torch.int32, mask_heads * nb + 1)
+    _cuda_tensor(col_idx, "col_idx", torch.int32)
+    _check(lib.lva_window_transposed_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, n, d, window,
+                                          block_size, _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), mask_heads,
+                                          ctypes.c_float(scale), ctypes.c_void_p(_stream(q.device))))
+    return o, lse
 
 
 def lva_broadcast_blocks(o, lse, block_size: int, query_src):

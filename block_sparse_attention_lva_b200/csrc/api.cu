@@ -180,7 +180,8 @@ static lva_status attn_common(const char* fn, const void* q, const void* k, cons
                               int block_size, const int32_t* row_ptr, const int32_t* col_idx,
                               int64_t col_len, int mask_heads, float scale, const int32_t* query_src,
                               int src_heads, void* o_raster, int T, int Hg, int Wg, int tile_t,
-                              int tile_h, int tile_w, cudaStream_t stream) {
+                              int tile_h, int tile_w, int gather_windows, int gather_window,
+                              cudaStream_t stream) {
   if (B < 0 || H < 1) return fail(LVA_ERR_INVALID_ARG, "%s: need B >= 0 and H >= 1", fn);
   if (d != 64 && d != 128) return fail(LVA_ERR_UNSUPPORTED, "%s: head dim must be 64 or 128", fn);
   if (block_size != 64 && block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "%s: block_size must be 64 or 128", fn);
@@ -212,7 +213,7 @@ static lva_status attn_common(const char* fn, const void* q, const void* k, cons
   if (err == nullptr) return fail(LVA_ERR_CUDA, "%s: cannot locate the device error word", fn);
   AttnArgs a{q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr,
              col_idx, col_len, mask_heads, scale, query_src, src_heads, err,
-             o_raster, T, Hg, Wg, tile_t, tile_h, tile_w};
+             o_raster, T, Hg, Wg, tile_t, tile_h, tile_w, gather_windows, gather_window};
   const char* why = "launch";
   cudaError_t e = launch_attn(a, stream, &why);
   if (e != cudaSuccess) return fail(LVA_ERR_CUDA, "%s: %s: %s", fn, why, cudaGetErrorString(e));
@@ -226,7 +227,7 @@ lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, vo
                                  cudaStream_t stream) {
   if (o == nullptr && B > 0) return fail(LVA_ERR_INVALID_ARG, "attn: null pointer");
   return attn_common("attn", q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr, col_idx,
-                     col_len, mask_heads, scale, query_src, src_heads, nullptr, 0, 0, 0, 0, 0, 0,
+                     col_len, mask_heads, scale, query_src, src_heads, nullptr, 0, 0, 0, 0, 0, 0, 0, 0,
                      stream);
 }
 
@@ -239,7 +240,28 @@ lva_status lva_block_sparse_attn_raster(const void* q, const void* k, const void
   if (o_raster == nullptr && B > 0) return fail(LVA_ERR_INVALID_ARG, "attn_raster: null pointer");
   return attn_common("attn_raster", q, k, v, nullptr, lse, B, H, n_pad, n_valid, d, block_size,
                      row_ptr, col_idx, col_len, mask_heads, scale, nullptr, 1, o_raster, T, Hg, Wg,
-                     tile_t, tile_h, tile_w, stream);
+                     tile_t, tile_h, tile_w, 0, 0, stream);
+}
+
+lva_status lva_window_transposed_attn(const void* q, const void* k, const void* v, void* o, float* lse,
+                                      int B, int H, int64_t n, int d, int window, int block_size,
+                                      const int32_t* row_ptr, const int32_t* col_idx, int64_t col_len,
+                                      int mask_heads, float scale, cudaStream_t stream) {
+  if (window < 1 || n <= 0 || n % window != 0)
+    return fail(LVA_ERR_INVALID_ARG, "window_attn: n must be a positive multiple of window");
+  const int64_t m = n / window;
+  if (block_size != 64 && block_size != 128)
+    return fail(LVA_ERR_UNSUPPORTED, "window_attn: block_size must be 64 or 128");
+  if (m % block_size != 0)
+    return fail(LVA_ERR_INVALID_ARG, "window_attn: the window count n / window must be a multiple of block_size");
+  if (int64_t(B) * H * m >= (int64_t(1) << 31))
+    return fail(LVA_ERR_UNSUPPORTED, "window_attn: B*H*(n/window) must be < 2^31");
+  if (o == nullptr && B > 0) return fail(LVA_ERR_INVALID_ARG, "window_attn: null pointer");
+  // O goes to the original order through the raster epilogue: the window transpose is the
+  // tile order of the grid (1, m, window) with tiles (1, m, 1).
+  return attn_common("window_attn", q, k, v, nullptr, lse, B, H, n, n, d, block_size, row_ptr, col_idx,
+                     col_len, mask_heads, scale, nullptr, 1, o, 1, int(m), window, 1, int(m), 1, int(m),
+                     window, stream);
 }
 
 lva_status lva_broadcast_blocks(void* o, float* lse, int B, int H, int64_t n_pad, int d, int block_size,

@@ -69,6 +69,9 @@ struct AttnParams {
   __nv_bfloat16* o;                // tile order [planes, n_pad, D], or
   __nv_bfloat16* o_raster;         // when set: raster order [planes, n_valid, D] (o unused)
   Grid3 grid;                      // latent grid and tile of the raster order
+  int gather_windows;              // 0: rows are plane-major [planes, n_pad, D]; m > 0: q, k,
+                                   // v hold m windows per plane and row k of the
+                                   // window-transposed order is read through a 3D map
   float* lse;
   const int32_t* query_src;        // NULL or [src_heads, nb]: blocks copied from an anchor
   int src_heads;
@@ -190,6 +193,19 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) LVA_TRACE_AT(20, 0);
 
+  // TMA load of the 64-element column chunk c of the rows [k0, k0 + box) of this plane:
+  // plane-major rows, or (window-gather maps) row k = pos * m + a of the window-transposed
+  // order, which is row a * w + pos of the input: coordinates (c * 64, pos, plane * m + a).
+  auto load_rows = [&](uint32_t dst, const void* tmap, int c, int64_t k0, uint32_t bar) {
+    if (p.gather_windows == 0) {
+      tma_load_2d(dst, tmap, c * 64, int32_t(plane * p.n_pad + k0), bar);
+    } else {
+      const int64_t m = p.gather_windows;
+      const int64_t pos = k0 / m;
+      tma_load_3d(dst, tmap, c * 64, int32_t(pos), int32_t(plane * m + (k0 - pos * m)), bar);
+    }
+  };
+
   // One TMA producer loop: tile t of `n` goes to slot t % ST of a ring whose slots are
   // released by `empty` barriers; after an abort, waits for the loads already issued.
   auto produce = [&](const void* tmap, uint32_t ring, int ST, uint32_t full0, uint32_t empty0, int code) {
@@ -200,11 +216,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         *abort_flag = 1; report_fault(p.err, 5, code); break;
       }
       const int32_t j = __ldg(p.col_idx + start + t);
-      const int32_t kv_row = int32_t(plane * p.n_pad + int64_t(j) * BN);
       mbar_arrive_expect_tx(full0 + 8u * s, C::KV_BYTES);
       LVA_TRACE_AT(code == 1 ? 14 : 15, t);
       for (int c = 0; c < D / 64; ++c)
-        tma_load_2d(ring + s * C::KV_BYTES + c * BN * 128, tmap, c * 64, kv_row, full0 + 8u * s);
+        load_rows(ring + s * C::KV_BYTES + c * BN * 128, tmap, c, int64_t(j) * BN, full0 + 8u * s);
       issued = t + 1;
     }
     if (*abort_flag)
@@ -216,9 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     // ------------------------------------------------------------ TMA producer: Q, K
     if (lane == 0 && n > 0) {
       tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k);
-      const int32_t q_row = int32_t(plane * p.n_pad + int64_t(i) * BN);
       mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
-      for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * BM * 128, &tm_q, c * 64, q_row, bar_q);
+      for (int c = 0; c < D / 64; ++c) load_rows(sQ + c * BM * 128, &tm_q, c, int64_t(i) * BN, bar_q);
       produce(&tm_k, sK, C::KST, bar_k_full(0), bar_k_empty(0), 1);
       if (*abort_flag) mbar_wait(bar_q, 0, never);
     }
@@ -507,43 +521,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// 2D view [rows, d] of a bf16 [B, H, n_pad, d] tensor; box = 64 elements x box_rows.
-bool make_map(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(d) * 2};
-  const cuuint32_t box[2] = {64u, cuuint32_t(box_rows)};
-  const cuuint32_t estr[2] = {1u, 1u};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, int BN>
 cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why) {
   using C = Cfg<D, BN>;
   const int64_t rows = int64_t(a.B) * a.H * a.n_pad;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, a.q, rows, D, BM) || !make_map(&tk, a.k, rows, D, BN) ||
-      !make_map(&tv, a.v, rows, D, BN)) {
+  bool maps_ok;
+  if (a.gather_windows == 0) {
+    maps_ok = make_rows_map(&tq, a.q, rows, D, BM) && make_rows_map(&tk, a.k, rows, D, BN) &&
+              make_rows_map(&tv, a.v, rows, D, BN);
+  } else {
+    const int64_t planes = int64_t(a.B) * a.H;
+    maps_ok = make_window_gather_map(&tq, a.q, planes, a.gather_windows, a.gather_window, D, BM) &&
+              make_window_gather_map(&tk, a.k, planes, a.gather_windows, a.gather_window, D, BN) &&
+              make_window_gather_map(&tv, a.v, planes, a.gather_windows, a.gather_window, D, BN);
+  }
+  if (!maps_ok) {
     *why = "cuTensorMapEncodeTiled failed or is unavailable";
     return cudaErrorInvalidValue;
   }
@@ -570,6 +563,7 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   p.o_raster = static_cast<__nv_bfloat16*>(a.o_raster);
   p.grid = Grid3{uint32_t(a.T), uint32_t(a.Hg), uint32_t(a.Wg), uint32_t(a.tt), uint32_t(a.th),
                  uint32_t(a.tw)};
+  p.gather_windows = a.gather_windows;
   p.lse = a.lse;
   p.query_src = a.query_src;
   p.src_heads = a.src_heads;

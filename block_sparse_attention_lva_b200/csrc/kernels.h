@@ -53,6 +53,8 @@ struct AttnArgs {
   int* err;  // device error word
   void* o_raster;            // NULL, or O in raster order [B, H, n_valid, d] instead of o
   int T, Hg, Wg, tt, th, tw; // latent grid and tile (used with o_raster)
+  int gather_windows;        // 0, or m: q, k, v are read window-transposed (see api.cu)
+  int gather_window;         // w, the tokens per window, with gather_windows
 };
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why);
 
@@ -111,6 +113,12 @@ constexpr int kSelectMaxBlocks = 4096;
 // 128-byte swizzle (from tmap.cu).  Returns false when the driver entry point is missing
 // or the encoding fails.
 bool make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows);
+
+// 3D tensor map over a bf16 [planes * windows, window, d] buffer, box of 64 elements x 1
+// position x box_rows windows: one box gathers the rows of box_rows consecutive windows at
+// one position, i.e. box_rows consecutive rows of the window-transposed order.
+bool make_window_gather_map(CUtensorMap* m, const void* base, int64_t planes, int windows, int window,
+                            int d, int box_rows);
 
 // Device error word of the current device (from api.cu).
 int* device_error_word();

@@ -237,18 +237,16 @@ class SquadTwoPass:
 
     Local pass: softmax attention inside consecutive windows of ``window`` tokens (the window
     mask kind with unit = window, radius 0, no anchors: block-diagonal).  Global pass: the
-    tokens at the same position of every window attend each other; the window transpose
-    that makes those groups contiguous is the tile reorder of the grid (1, m, window) with
-    tiles (1, m, 1), m = n / window.  The local output is the global pass's value stream:
+    tokens at the same position of every window attend each other, with the local output as
+    the value stream:
 
-        O = T^-1( Attn_G( T(Q), T(K), T(Attn_L(Q, K, V)) ) )
+        O[a*w + p] = softmax over a' of (q_{a*w+p} . k_{a'*w+p}) O_L[a'*w + p]
 
-    (T^-1 is applied by the global pass's epilogue, which stores each row at its position in
-    the original order.)
-
-    ``window`` and ``m`` must be multiples of ``block_size``; inputs are [B, H, n, d] bf16 in
-    the order whose consecutive tokens form the windows (e.g. after the spatiotemporal tile
-    reorder).
+    The global pass runs on the window-transposed order (position-major, row p*m + a) without
+    materialising it: ``lva_window_transposed_attn`` gathers those rows through 3D tensor maps
+    and stores O back in the input order.  ``window`` and ``m = n / window`` must be multiples
+    of ``block_size``; inputs are [B, H, n, d] bf16 in the order whose consecutive tokens form
+    the windows (e.g. after the spatiotemporal tile reorder).
     """
 
     def __init__(self, B, H, n, d, window, block_size=128, scale=None, device="cuda"):
@@ -261,13 +259,13 @@ class SquadTwoPass:
         kw = dict(device=self.device)
         shape = (B, H, n, d)
         self.o_local = torch.empty(shape, dtype=torch.bfloat16, **kw)
-        self.qk_t = torch.empty((2,) + shape, dtype=torch.bfloat16, **kw)     # transposed Q, K
-        self.o_local_t = torch.empty(shape, dtype=torch.bfloat16, **kw)
         self.o = torch.empty(shape, dtype=torch.bfloat16, **kw)
         self.lse_local = torch.empty((B, H, n), dtype=torch.float32, **kw)
-        self.lse_global_t = torch.empty((B, H, n), dtype=torch.float32, **kw)
+        self.lse_global_t = torch.empty((B, H, n), dtype=torch.float32, **kw)   # transposed order
         nb = n // block_size
         self.csr = {}
+        # local: groups of `window` consecutive tokens; global: groups of m consecutive rows of
+        # the transposed order (one position across all windows)
         for name, unit in (("local", window), ("global", self.m)):
             p = lb.MaskParams(lb.LVA_MASK_WINDOW_ANCHOR, n, n, block_size, 1, unit, 0, 0, 0)
             row_ptr = torch.empty(nb + 1, dtype=torch.int32, **kw)
@@ -275,29 +273,14 @@ class SquadTwoPass:
             nnz = torch.empty(1, dtype=torch.int32, **kw)
             lb.lva_build_block_mask(p, None, row_ptr, col_idx, nnz)
             self.csr[name] = (row_ptr, col_idx)
-        self.grid, self.tile = (1, self.m, window), (1, self.m, 1)
-
-    def _transpose(self, src, dst, planes, inverse=False):
-        lb.lva_reorder_tokens(src.reshape(planes, self.n, self.d), dst.reshape(planes, self.n, self.d),
-                              self.grid, self.tile, self.n, inverse=inverse)
 
     def __call__(self, q, k, v):
-        P = self.B * self.H
         rp, ci = self.csr["local"]
         lb.lva_block_sparse_attn(q, k, v, self.o_local, self.lse_local, self.n, self.block_size, rp, ci, 1,
                                  self.scale)
-        if VideoBlockSparseAttention._stacked(q, k, v):
-            base = q.reshape(-1)
-            qk = torch.as_strided(base, (2 * P, self.n, self.d), (self.n * self.d, self.d, 1))
-            self._transpose(qk, self.qk_t, 2 * P)
-        else:
-            self._transpose(q, self.qk_t[0], P)
-            self._transpose(k, self.qk_t[1], P)
-        self._transpose(self.o_local, self.o_local_t, P)
         rp, ci = self.csr["global"]
-        # The inverse window transpose is the raster store of the global pass's epilogue.
-        lb.lva_block_sparse_attn_raster(self.qk_t[0], self.qk_t[1], self.o_local_t, self.o, self.lse_global_t,
-                                        self.n, self.block_size, rp, ci, 1, self.scale, self.grid, self.tile)
+        lb.lva_window_transposed_attn(q, k, self.o_local, self.o, self.lse_global_t, self.window,
+                                      self.block_size, rp, ci, 1, self.scale)
         return self.o
 
 

@@ -205,6 +205,30 @@ lva_status lva_block_sparse_attn_raster(const void* q, const void* k, const void
                                         int tile_w, cudaStream_t stream);
 
 /*
+ * lva_window_transposed_attn -- block-sparse attention across windows, without a transpose.
+ *
+ * SQuad page ("SQuad: Sub-Quadratic Attention Distillation for Efficient Video Generation"),
+ * technical summary section 1: the global pass of the two-stage operator mixes the tokens at
+ * the same relative position of every window.  With windows of w tokens (m = n / w windows),
+ * token a*w + p is position p of window a; the window-transposed order lists position-major,
+ *   row k = p*m + a of the transposed order  <->  token a*w + p of the input,
+ * so each group of m consecutive transposed rows is one position across all windows.  This
+ * call computes lva_block_sparse_attn on the transposed order (CSR over its blocks, same
+ * definition and arithmetic) while reading q, k, v in the input order through 3D tensor
+ * maps (a box gathers the rows of consecutive windows at one position), and stores O back in
+ * the input order.  LSE is in the transposed order.
+ *
+ * q, k, v, o: device bf16 [B, H, n, d] in the input order, 16-byte aligned (o written);
+ * lse: device fp32 [B, H, n].  n = m*w with m a multiple of block_size (a block never spans
+ * two positions); no padding (n_valid = n).  Other arguments and errors as for
+ * lva_block_sparse_attn (no repetitive-head maps).
+ */
+lva_status lva_window_transposed_attn(const void* q, const void* k, const void* v, void* o, float* lse,
+                                      int B, int H, int64_t n, int d, int window, int block_size,
+                                      const int32_t* row_ptr, const int32_t* col_idx, int64_t col_len,
+                                      int mask_heads, float scale, cudaStream_t stream);
+
+/*
  * lva_broadcast_blocks -- fill the query blocks of repetitive heads from their anchors.
  *
  * CalibAtt page ("Accelerating Text-to-Video Generation with Calibrated Sparse Attention",

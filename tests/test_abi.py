@@ -115,3 +115,16 @@ def test_calibration_argument_checks_fail_before_launch():
     assert agg(0, 16, 0.5) == 1
     assert agg(2, 16, 1.5) == 1
     assert agg(2, 0, 0.5) == 0
+
+
+def test_window_transposed_attn_argument_checks():
+    from block_sparse_attention_lva_b200._binding import lib
+    vp = ctypes.c_void_p(64)
+    call = lambda n, w, bs=128, d=128: lib.lva_window_transposed_attn(
+        vp, vp, vp, vp, vp, 1, 2, n, d, w, bs, vp, vp, 4, 1, ctypes.c_float(0.1), None)
+    assert call(32768, 300) == 1            # n not a multiple of the window
+    assert call(32768, 512) == 1            # m = 64 windows: not a multiple of the block
+    assert call(32768, 256, bs=32) == 2     # unsupported block size
+    assert call(32768, 256, d=96) == 2      # unsupported head dim
+    assert lib.lva_window_transposed_attn(vp, vp, vp, None, vp, 1, 2, 32768, 128, 256, 128, vp, vp, 4, 1,
+                                          ctypes.c_float(0.1), None) == 1
