@@ -536,7 +536,7 @@ def run_report(args):
         print(json.dumps({"report": "squad_two_pass", "heads": H, "tokens": n, "window": win,
                           "active_pairs": pairs, "ms": ms, "tflops": flops / ms / 1e9,
                           "frac_of_burst": flops / ms / 1e9 / burst,
-                          "note": "2 attention launches + 2 transpose launches (Q/K stacked, local O); the inverse transpose is the global pass epilogue; FLOPs of both passes"}),
+                          "note": "2 attention launches, no transposes: the global pass gathers the window-transposed rows through 3D tensor maps and stores O in the input order; FLOPs of both passes"}),
               flush=True)
         del qkv, op
         torch.cuda.empty_cache()
