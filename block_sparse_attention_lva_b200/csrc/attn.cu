@@ -69,6 +69,7 @@ struct AttnParams {
   __nv_bfloat16* o;                // tile order [planes, n_pad, D], or
   __nv_bfloat16* o_raster;         // when set: raster order [planes, n_valid, D] (o unused)
   Grid3 grid;                      // latent grid and tile of the raster order
+  int64_t items;                   // (plane, query block) work items: planes * nb
   int gather_windows;              // 0: rows are plane-major [planes, n_pad, D]; m > 0: q, k,
                                    // v hold m windows per plane and row k of the
                                    // window-transposed order is read through a 3D map
@@ -88,10 +89,13 @@ struct Cfg {
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
   // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2],
-  // s_free[2], p_full[2], o_done[2] (P*V done, per P buffer), final (Q K^T), final (P V)
+  // s_free[2], p_full[2], o_done[2] (P*V done, per P buffer), final (Q K^T), final (P V),
+  // q_empty (an item's Q K^T done: Q may be replaced), o_free (an item's O read: P V may
+  // start the next item)
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST, B_VE = B_VF + VST,
                        B_SF = B_VE + VST, B_SE = B_SF + 2, B_P = B_SE + 2, B_O = B_P + 2,
-                       B_FIN = B_O + 2, B_FIN_PV = B_FIN + 1, NUM_BARS = B_FIN_PV + 1;
+                       B_FIN = B_O + 2, B_FIN_PV = B_FIN + 1, B_QE = B_FIN_PV + 1, B_OF = B_QE + 1,
+                       NUM_BARS = B_OF + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // At least 120 KB so that one CTA (and one 512-column TMEM allocation) is resident per SM.
   static constexpr int SMEM_RAW = OFF_MISC + 16;
@@ -124,7 +128,7 @@ __device__ __forceinline__ int csr_row(const AttnParams& p, int64_t row, int32_t
   return b - a;
 }
 
-template <int D, int BN>
+template <int D, int BN, int KPC>
 __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -149,6 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   auto bar_o_done = [&](int b) { return bar0 + 8u * (C::B_O + b); };
   const uint32_t bar_final = bar0 + 8u * C::B_FIN;
   const uint32_t bar_final_pv = bar0 + 8u * C::B_FIN_PV;
+  const uint32_t bar_q_empty = bar0 + 8u * C::B_QE;
+  const uint32_t bar_o_free = bar0 + 8u * C::B_OF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   // Stays zero: the drain waits after an abort are bounded by time alone.
@@ -156,22 +162,34 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Work item: plane-major, query block fastest, so neighbouring CTAs share one head's K/V.
-  const int64_t item = blockIdx.x;
-  const int64_t plane = item / p.nb;
-  const int i = int(item - plane * p.nb);
-  const int h = int(plane % p.H);
-  // Blocks of repetitive heads that take an anchor's output are not computed here.
-  if (p.query_src != nullptr &&
-      __ldg(p.query_src + int64_t(p.src_heads == 1 ? 0 : h) * p.nb + i) != i)
-    return;
-  const int64_t csr = int64_t(p.mask_heads == 1 ? 0 : h) * p.nb + i;
-  int32_t start;
-  bool bad;
-  const int n = csr_row(p, csr, start, bad);
+  // Work items: (plane, query block), plane-major with the query block fastest.  The CTA
+  // takes a run of consecutive items (below).  Every role walks the same items; pipeline
+  // positions T count key blocks over all items of this CTA, so ring slots, S/P buffers and
+  // their barrier phases simply continue from one item to the next, and the next item's Q
+  // load and first Q K^T overlap the current item's epilogue.
+  const int items = int(p.items);               // < 2^31: B*H*n_pad < 2^31 is enforced
+  // This CTA's items: a run of consecutive query blocks (same plane, overlapping key lists,
+  // so their K/V tiles stay in L2); CTAs are launched in item order.
+  const int it_begin = int(blockIdx.x) * KPC;
+  const int it_end = it_begin + KPC < items ? it_begin + KPC : items;
+  // Per item: whether it is computed here, its CSR row start and length (every warp derives
+  // the same values from the same memory; a corrupt row counts as empty).
+  struct Item { int plane; int i; int32_t start; int n; bool skip; bool bad; };
+  auto item_at = [&](int it) -> Item {
+    Item r;
+    r.plane = it / p.nb;
+    r.i = it - r.plane * p.nb;
+    const int h = r.plane % p.H;
+    r.skip = p.query_src != nullptr &&
+             __ldg(p.query_src + int64_t(p.src_heads == 1 ? 0 : h) * p.nb + r.i) != r.i;
+    r.n = 0; r.start = 0; r.bad = false;
+    if (!r.skip) r.n = csr_row(p, int64_t(p.mask_heads == 1 ? 0 : h) * p.nb + r.i, r.start, r.bad);
+    return r;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
+    mbar_init(bar_q_empty, 1);
     for (int s = 0; s < C::KST; ++s) { mbar_init(bar_k_full(s), 1); mbar_init(bar_k_empty(s), 1); }
     for (int s = 0; s < C::VST; ++s) { mbar_init(bar_v_full(s), 1); mbar_init(bar_v_empty(s), 1); }
     for (int b = 0; b < 2; ++b) {
@@ -180,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       mbar_init(bar_p_full(b), kSoftmaxWarps);
       mbar_init(bar_o_done(b), 1);
     }
+    mbar_init(bar_o_free, kSoftmaxWarps);
     mbar_init(bar_final, 1);
     mbar_init(bar_final_pv, 1);
     *abort_flag = 0;
@@ -193,10 +212,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   const uint32_t tmem = *tmem_slot;
   if (threadIdx.x == 0) LVA_TRACE_AT(20, 0);
 
-  // TMA load of the 64-element column chunk c of the rows [k0, k0 + box) of this plane:
+  // TMA load of the 64-element column chunk c of the rows [k0, k0 + box) of a plane:
   // plane-major rows, or (window-gather maps) row k = pos * m + a of the window-transposed
   // order, which is row a * w + pos of the input: coordinates (c * 64, pos, plane * m + a).
-  auto load_rows = [&](uint32_t dst, const void* tmap, int c, int64_t k0, uint32_t bar) {
+  auto load_rows = [&](uint32_t dst, const void* tmap, int c, int64_t plane, int64_t k0, uint32_t bar) {
     if (p.gather_windows == 0) {
       tma_load_2d(dst, tmap, c * 64, int32_t(plane * p.n_pad + k0), bar);
     } else {
@@ -206,71 +225,97 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     }
   };
 
-  // One TMA producer loop: tile t of `n` goes to slot t % ST of a ring whose slots are
-  // released by `empty` barriers; after an abort, waits for the loads already issued.
-  auto produce = [&](const void* tmap, uint32_t ring, int ST, uint32_t full0, uint32_t empty0, int code) {
-    int issued = 0;
-    for (int t = 0; t < n; ++t) {
-      const int s = t % ST;
-      if (t >= ST && !mbar_wait(empty0 + 8u * s, ((t / ST) - 1) & 1, abort_flag)) {
-        *abort_flag = 1; report_fault(p.err, 5, code); break;
+  // A TMA producer: key block T (over all items) goes to slot T % ST of a ring whose slots
+  // are released by `empty` barriers; after an abort it waits for the loads still in flight.
+  auto produce = [&](const void* tmap, uint32_t ring, int ST, uint32_t full0, uint32_t empty0, int code,
+                     bool with_q) {
+    uint32_t T = 0;         // key blocks issued so far
+    int nq = 0;             // Q tiles issued so far
+    for (int it = it_begin; it < it_end; ++it) {
+      if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;     // one decision for the warp
+      const Item w = item_at(it);
+      if (w.n == 0) continue;
+      if (lane == 0) {
+        if (with_q) {
+          // Q is single-buffered: the previous item's Q K^T must have completed.
+          if (nq > 0 && !mbar_wait(bar_q_empty, (nq - 1) & 1, abort_flag)) {
+            *abort_flag = 1; report_fault(p.err, 5, 8);
+          } else {
+            mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
+            for (int c = 0; c < D / 64; ++c)
+              load_rows(sQ + c * BM * 128, &tm_q, c, w.plane, int64_t(w.i) * BN, bar_q);
+            ++nq;
+          }
+        }
+        for (int t = 0; t < w.n && !*abort_flag; ++t, ++T) {
+          const int s = int(T % ST);
+          if (T >= ST && !mbar_wait(empty0 + 8u * s, int((T / ST) - 1) & 1, abort_flag)) {
+            *abort_flag = 1; report_fault(p.err, 5, code); break;
+          }
+          const int32_t j = __ldg(p.col_idx + w.start + t);
+          mbar_arrive_expect_tx(full0 + 8u * s, C::KV_BYTES);
+          for (int c = 0; c < D / 64; ++c)
+            load_rows(ring + s * C::KV_BYTES + c * BN * 128, tmap, c, w.plane, int64_t(j) * BN, full0 + 8u * s);
+        }
       }
-      const int32_t j = __ldg(p.col_idx + start + t);
-      mbar_arrive_expect_tx(full0 + 8u * s, C::KV_BYTES);
-      LVA_TRACE_AT(code == 1 ? 14 : 15, t);
-      for (int c = 0; c < D / 64; ++c)
-        load_rows(ring + s * C::KV_BYTES + c * BN * 128, tmap, c, int64_t(j) * BN, full0 + 8u * s);
-      issued = t + 1;
+      __syncwarp();
     }
-    if (*abort_flag)
-      for (int t = (issued > ST ? issued - ST : 0); t < issued; ++t)
-        mbar_wait(full0 + 8u * (t % ST), (t / ST) & 1, never);
+    if (lane == 0 && *abort_flag) {
+      for (uint32_t u = (T > uint32_t(ST) ? T - ST : 0); u < T; ++u)
+        mbar_wait(full0 + 8u * int(u % ST), int(u / ST) & 1, never);
+      if (with_q && nq > 0) mbar_wait(bar_q, (nq - 1) & 1, never);
+    }
   };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer: Q, K
-    if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k);
-      mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
-      for (int c = 0; c < D / 64; ++c) load_rows(sQ + c * BM * 128, &tm_q, c, int64_t(i) * BN, bar_q);
-      produce(&tm_k, sK, C::KST, bar_k_full(0), bar_k_empty(0), 1);
-      if (*abort_flag) mbar_wait(bar_q, 0, never);
-    }
+    if (lane == 0) { tma_prefetch_desc(&tm_q); tma_prefetch_desc(&tm_k); }
+    produce(&tm_k, sK, C::KST, bar_k_full(0), bar_k_empty(0), 1, true);
   } else if (warp == kVWarp) {
     // ------------------------------------------------------------ TMA producer: V
-    if (lane == 0 && n > 0) {
-      tma_prefetch_desc(&tm_v);
-      produce(&tm_v, sV, C::VST, bar_v_full(0), bar_v_empty(0), 6);
-    }
+    if (lane == 0) tma_prefetch_desc(&tm_v);
+    produce(&tm_v, sV, C::VST, bar_v_full(0), bar_v_empty(0), 6, false);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer: S = Q K^T
-    // S(t+2) is issued as soon as the softmax has read S(t) (same S buffer).  O += P V is
+    // S(T+2) is issued as soon as the softmax has read S(T) (same S buffer).  O += P V is
     // issued by its own warp, so neither issue stream waits behind the other's barriers;
     // the two write disjoint TMEM columns and read disjoint shared memory.  Descriptors are
     // built once; an MMA only adds a byte offset / 16 to the start-address field (shared
     // addresses stay below 2^18 bytes, so the 14-bit field never carries).
-    if (lane == 0 && n > 0) {
-      const uint64_t q_desc = smem_desc_sw128(sQ, 16, 1024);
-      const uint64_t k_desc = smem_desc_sw128(sK, 16, 1024);
-      bool ok = mbar_wait(bar_q, 0, abort_flag);
-      bool any_mma = false;
-      for (int t = 0; ok && t < n; ++t) {
-        const int s = t % C::KST, b = t & 1;
-        if (!mbar_wait(bar_k_full(s), (t / C::KST) & 1, abort_flag)) { ok = false; break; }
-        if (t >= 2 && !mbar_wait(bar_s_free(b), ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        LVA_TRACE_AT(0, t);
-        const uint64_t ks = k_desc + uint64_t((s * C::KV_BYTES) >> 4);
-        const uint32_t s_tm = tmem + C::TM_S + 128 * b;
+    const uint64_t q_desc = smem_desc_sw128(sQ, 16, 1024);
+    const uint64_t k_desc = smem_desc_sw128(sK, 16, 1024);
+    bool ok = true, any_mma = false;
+    uint32_t T = 0;
+    int nq = 0;
+    for (int it = it_begin; ok && it < it_end; ++it) {
+      const Item w = item_at(it);
+      if (w.n == 0) continue;
+      if (lane == 0) {
+        ok = mbar_wait(bar_q, nq & 1, abort_flag);
+        for (int t = 0; ok && t < w.n; ++t, ++T) {
+          const int s = int(T % C::KST), b = int(T & 1);
+          if (!mbar_wait(bar_k_full(s), int(T / C::KST) & 1, abort_flag)) { ok = false; break; }
+          if (T >= 2 && !mbar_wait(bar_s_free(b), int((T >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          LVA_TRACE_AT(0, nq == 0 ? t : 64);
+          const uint64_t ks = k_desc + uint64_t((s * C::KV_BYTES) >> 4);
+          const uint32_t s_tm = tmem + C::TM_S + 128 * b;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_f16_ss(s_tm, q_desc + uint64_t(((kk / 4) * BM * 128 + (kk % 4) * 32) >> 4),
-                      ks + uint64_t(((kk / 4) * BN * 128 + (kk % 4) * 32) >> 4), C::IDESC_QK,
-                      kk > 0 ? 1u : 0u);
-        umma_commit(bar_s_full(b));
-        umma_commit(bar_k_empty(s));
-        any_mma = true;
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_f16_ss(s_tm, q_desc + uint64_t(((kk / 4) * BM * 128 + (kk % 4) * 32) >> 4),
+                        ks + uint64_t(((kk / 4) * BN * 128 + (kk % 4) * 32) >> 4), C::IDESC_QK,
+                        kk > 0 ? 1u : 0u);
+          umma_commit(bar_s_full(b));
+          umma_commit(bar_k_empty(s));
+          any_mma = true;
+        }
+        // Q may be replaced once this item's Q K^T MMAs have completed.
+        if (ok) umma_commit(bar_q_empty);
+        ++nq;
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    if (lane == 0) {
       if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 2); }
       if (any_mma) {
         // Drain: every MMA issued by this thread completes before TMEM is released.
@@ -280,26 +325,39 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     }
   } else if (warp == kPVWarp) {
     // ------------------------------------------------------------ MMA issuer: O += P V
-    // O += P(t) V_t as soon as P(t) is in TMEM and V_t has landed; P is the TMEM A operand.
-    if (lane == 0 && n > 0) {
-      const uint64_t v_desc = smem_desc_sw128(sV, BN * 128, 1024);
-      bool ok = true, any_mma = false;
-      for (int t = 0; ok && t < n; ++t) {
-        const int s = t % C::VST, b = t & 1;
-        if (!mbar_wait(bar_p_full(b), (t >> 1) & 1, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(bar_v_full(s), (t / C::VST) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        LVA_TRACE_AT(1, t);
-        const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
-        const uint32_t p_tm = tmem + C::TM_P + 64 * b;
+    // O += P(T) V_T as soon as P(T) is in TMEM and V_T has landed; P is the TMEM A operand.
+    // An item's first P V overwrites O, so it waits until the softmax warps have read the
+    // previous item's O in their epilogue.
+    const uint64_t v_desc = smem_desc_sw128(sV, BN * 128, 1024);
+    bool ok = true, any_mma = false;
+    uint32_t T = 0;
+    int nq = 0;
+    for (int it = it_begin; ok && it < it_end; ++it) {
+      const Item w = item_at(it);
+      if (w.n == 0) continue;
+      if (lane == 0) {
+        if (nq > 0) ok = mbar_wait(bar_o_free, (nq - 1) & 1, abort_flag);
+        for (int t = 0; ok && t < w.n; ++t, ++T) {
+          const int s = int(T % C::VST), b = int(T & 1);
+          if (!mbar_wait(bar_p_full(b), int(T >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(bar_v_full(s), int(T / C::VST) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          LVA_TRACE_AT(1, nq == 0 ? t : 64);
+          const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
+          const uint32_t p_tm = tmem + C::TM_P + 64 * b;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          umma_f16_ts(tmem + C::TM_O, p_tm + kk * 8, vs + uint64_t((kk * 16 * 128) >> 4), C::IDESC_PV,
-                      (t > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar_v_empty(s));
-        umma_commit(bar_o_done(b));
-        any_mma = true;
+          for (int kk = 0; kk < BN / 16; ++kk)
+            umma_f16_ts(tmem + C::TM_O, p_tm + kk * 8, vs + uint64_t((kk * 16 * 128) >> 4), C::IDESC_PV,
+                        (t > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar_v_empty(s));
+          umma_commit(bar_o_done(b));
+          any_mma = true;
+        }
+        ++nq;
       }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    if (lane == 0) {
       if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 7); }
       if (any_mma) {
         umma_commit(bar_final_pv);
@@ -318,199 +376,218 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     const int row = quarter * 32 + sel * 16 + (lane & 15);   // row of the 128-row tile
     const uint32_t lane_off = uint32_t(quarter * 32 + sel * 16) << 16;
     const float c = p.scale_log2;                 // scores -> log2 units
-    float m_ref = -INFINITY;                      // running max in log2 units (lazy)
-    float l = 0.f;                                // this half's share of the row sum
     bool ok = true;
     const bool tr = (quarter == 2 && sel == 0 && lane == 0);
-    if (bad && threadIdx.x == kSoftmaxWarp0 * 32) report_fault(p.err, 1, int(csr & 0x7fffffff));
-    int32_t jn = n > 0 ? __ldg(p.col_idx + start) : 0;
+    uint32_t T = 0;
+    int nq = 0;
+    for (int it = it_begin; ok && it < it_end; ++it) {
+      const Item w = item_at(it);
+      if (w.skip) continue;
+      const int n = w.n;
+      if (w.bad && warp == kSoftmaxWarp0 && lane == 0)
+        report_fault(p.err, 1, (p.mask_heads == 1 ? 0 : w.plane % p.H) * p.nb + w.i);
+      float m_ref = -INFINITY;                    // running max in log2 units (lazy)
+      float l = 0.f;                              // this half's share of the row sum
+      int32_t jn = n > 0 ? __ldg(p.col_idx + w.start) : 0;
 
-    for (int t = 0; t < n; ++t) {
-      const int b = t & 1;
-      const int32_t j = jn;
-      if (t + 1 < n) jn = __ldg(p.col_idx + start + t + 1);
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), (t >> 1) & 1, abort_flag))) { ok = false; break; }
-      tc_fence_after();
-      if (tr) LVA_TRACE_AT(2, t);
-      uint32_t sr[HALF];
+      for (int t = 0; t < n; ++t, ++T) {
+        const int b = int(T & 1);
+        const int32_t j = jn;
+        if (t + 1 < n) jn = __ldg(p.col_idx + w.start + t + 1);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T >> 1) & 1, abort_flag))) { ok = false; break; }
+        tc_fence_after();
+        if (tr && nq == 0) LVA_TRACE_AT(2, t);
+        uint32_t sr[HALF];
 #pragma unroll
-      for (int q = 0; q < HALF / 32; ++q)
-        tmem_ld_16x2_32<HALF>(tmem + lane_off + C::TM_S + 128 * b + q * 32,
-                              *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_s_free(b));
-      if (tr) LVA_TRACE_AT(3, t);
-
-      // Real keys of this half (only the block holding the sequence end is partial).  The
-      // choice of path is made for the whole warp: the exponential loop below issues
-      // warp-collective TMEM stores, and the two halves of a row can differ at the end.
-      const int64_t valid = p.n_valid - int64_t(j) * BN - hf * HALF;
-      const bool full = __all_sync(0xffffffffu, valid >= HALF);
-      float mx;
-      if (full) {
-        // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (3-input max, 4 chains)
-        float m4[4];
-        if (c >= 0.f) {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
-#pragma unroll
-          for (int e = 0; e < HALF / 2; ++e)
-            m4[e & 3] = fmax3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
-          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 4; ++e) m4[e] = INFINITY;
-#pragma unroll
-          for (int e = 0; e < HALF / 2; ++e)
-            m4[e & 3] = fmin3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
-          mx = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3])) * c;
-        }
-      } else {
-        mx = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < HALF; ++e)
-          if (e < valid) mx = fmaxf(mx, __uint_as_float(sr[e]) * c);
-      }
-      // Row max over both halves (lanes t and t ^ 16 hold one row).
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-      const float m_old = m_ref;
-      if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
-      const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // P_b was last read by O += P(t-2) V; wait for it before any part of P(t) is stored.
-      // Each P buffer has its own completion barrier, so the wait never aliases an older
-      // phase.  (Almost always complete by now: P(t-2) V was issued a block earlier.)
-      if (t >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), ((t >> 1) - 1) & 1, abort_flag))) {
-        ok = false; break;
-      }
-      tc_fence_after();
-      const uint32_t p_tm = tmem + lane_off + C::TM_P + 64 * b;
-      float r4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[HALF / 2];
-      if (full) {
-        // Pairs of elements with packed fp32 math; every fourth pair takes its exponentials
-        // on the FMA pipe, the rest on the MUFU (of 1/2, 1/3, 1/4 and none on the FMA pipe,
-        // 1/4 measured fastest).  With 64-key halves the first 16 pairs go to TMEM while the
-        // rest are computed.
-        const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
-        uint64_t acc[2] = {0ull, 0ull};
-#pragma unroll
-        for (int e = 0; e < HALF / 2; ++e) {
-          const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
-          uint64_t p2;
-          if (e % 4 == 3) {
-            p2 = exp2_poly_f2(x2);
+        for (int q = 0; q < HALF / 32; ++q)
+          tmem_ld_16x2_32<HALF>(tmem + lane_off + C::TM_S + 128 * b + q * 32,
+                                *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_s_free(b));
+        if (tr && nq == 0) LVA_TRACE_AT(3, t);
+        // Real keys of this half (only the block holding the sequence end is partial).  The
+        // choice of path is made for the whole warp: the exponential loop below issues
+        // warp-collective TMEM stores, and the two halves of a row can differ at the end.
+        const int64_t valid = p.n_valid - int64_t(j) * BN - hf * HALF;
+        const bool full = __all_sync(0xffffffffu, valid >= HALF);
+        float mx;
+        if (full) {
+          // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (3-input max, 4 chains)
+          float m4[4];
+          if (c >= 0.f) {
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
+  #pragma unroll
+            for (int e = 0; e < HALF / 2; ++e)
+              m4[e & 3] = fmax3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
+            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
           } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) m4[e] = INFINITY;
+  #pragma unroll
+            for (int e = 0; e < HALF / 2; ++e)
+              m4[e & 3] = fmin3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
+            mx = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3])) * c;
           }
-          acc[e & 1] = f2_add(acc[e & 1], p2);
-          float p0, p1;
-          f2_unpack(p2, p0, p1);
-          pk[e] = pack_bf16x2(p0, p1);
-          if constexpr (HALF == 64) {
-            if (e == 15) tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
-          }
-        }
-        if constexpr (HALF == 64) {
-          tmem_st_16x2_16<HALF / 2>(p_tm + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
         } else {
-          tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          mx = -INFINITY;
+  #pragma unroll
+          for (int e = 0; e < HALF; ++e)
+            if (e < valid) mx = fmaxf(mx, __uint_as_float(sr[e]) * c);
         }
-        float a0, a1, b0, b1;
-        f2_unpack(acc[0], a0, a1);
-        f2_unpack(acc[1], b0, b1);
-        r4[0] = a0; r4[1] = a1; r4[2] = b0; r4[3] = b1;
-      } else {
-#pragma unroll
-        for (int e = 0; e < HALF; e += 2) {
-          const float p0 = e < valid ? ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use)) : 0.f;
-          const float p1 = e + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use)) : 0.f;
-          r4[(e >> 1) & 3] += p0 + p1;
-          pk[e / 2] = pack_bf16x2(p0, p1);
-        }
-        // P half row (bf16 pairs) -> TMEM P_b, the A operand of O += P V.
-        if constexpr (HALF == 64) {
-          tmem_st_16x2_32<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-        } else {
-          tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
-        }
-      }
-      l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
-      if (tr) LVA_TRACE_AT(4, t);
-
-      // O was last written by O += P(t-1) V: rescale it (rarely) once that has completed,
-      // before P(t) is released to the P V issuer.
-      if (t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(b ^ 1), ((t - 1) >> 1) & 1, abort_flag))) {
+        // Row max over both halves (lanes t and t ^ 16 hold one row).
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_old = m_ref;
+        if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
+        const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        // P_b was last read by O += P(t-2) V; wait for it before any part of P(t) is stored.
+        // Each P buffer has its own completion barrier, so the wait never aliases an older
+        // phase.  (Almost always complete by now: P(t-2) V was issued a block earlier.)
+        if (T >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), int((T >> 1) - 1) & 1, abort_flag))) {
           ok = false; break;
         }
         tc_fence_after();
-        if (tr) LVA_TRACE_AT(5, t);
+        const uint32_t p_tm = tmem + lane_off + C::TM_P + 64 * b;
+        float r4[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[HALF / 2];
+        if (full) {
+          // Pairs of elements with packed fp32 math; every fourth pair takes its exponentials
+          // on the FMA pipe, the rest on the MUFU (of 1/2, 1/3, 1/4 and none on the FMA pipe,
+          // 1/4 measured fastest).  With 64-key halves the first 16 pairs go to TMEM while the
+          // rest are computed.
+          const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
+          uint64_t acc[2] = {0ull, 0ull};
+  #pragma unroll
+          for (int e = 0; e < HALF / 2; ++e) {
+            const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
+            uint64_t p2;
+            if (e % 4 == 3) {
+              p2 = exp2_poly_f2(x2);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            }
+            acc[e & 1] = f2_add(acc[e & 1], p2);
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            pk[e] = pack_bf16x2(p0, p1);
+            if constexpr (HALF == 64) {
+              if (e == 15) tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+            }
+          }
+          if constexpr (HALF == 64) {
+            tmem_st_16x2_16<HALF / 2>(p_tm + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
+          } else {
+            tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          }
+          float a0, a1, b0, b1;
+          f2_unpack(acc[0], a0, a1);
+          f2_unpack(acc[1], b0, b1);
+          r4[0] = a0; r4[1] = a1; r4[2] = b0; r4[3] = b1;
+        } else {
+  #pragma unroll
+          for (int e = 0; e < HALF; e += 2) {
+            const float p0 = e < valid ? ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use)) : 0.f;
+            const float p1 = e + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use)) : 0.f;
+            r4[(e >> 1) & 3] += p0 + p1;
+            pk[e / 2] = pack_bf16x2(p0, p1);
+          }
+          // P half row (bf16 pairs) -> TMEM P_b, the A operand of O += P V.
+          if constexpr (HALF == 64) {
+            tmem_st_16x2_32<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+          } else {
+            tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          }
+        }
+        l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
+        if (tr && nq == 0) LVA_TRACE_AT(4, t);
+
+        // O was last written by O += P(t-1) V: rescale it (rarely) once that has completed,
+        // before P(t) is released to the P V issuer.
+        if (t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(b ^ 1), int((T - 1) >> 1) & 1, abort_flag))) {
+            ok = false; break;
+          }
+          tc_fence_after();
+          if (tr && nq == 0) LVA_TRACE_AT(5, t);
+  #pragma unroll 1
+          for (int q = 0; q < DH / 32; ++q) {
+            uint32_t ov[32];
+            tmem_ld_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
+            tmem_wait_ld();
+  #pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_p_full(b));
+        if (tr && nq == 0) LVA_TRACE_AT(7, t);
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue of this item
+      const int64_t plane = w.plane;
+      const int i = w.i;
+      const int64_t grow = int64_t(i) * BN + row;           // row within the plane
+      const bool store = row < BN && grow < p.n_pad;
+      // O row destination: tile order, or (fused inverse reorder) the row's raster position;
+      // padding rows have no raster position and are not written then.
+      __nv_bfloat16* orow;
+      bool store_o = store;
+      if (p.o_raster != nullptr) {
+        store_o = store && grow < p.n_valid;
+        const uint32_t raster = store_o ? tile_order_to_raster(uint32_t(grow), p.grid) : 0u;
+        orow = p.o_raster + (plane * p.n_valid + int64_t(raster)) * D + hf * DH;
+      } else {
+        orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
+      }
+      const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
+      const bool have = n > 0 && l_row > 0.f;
+      const float inv_l = have ? 1.f / l_row : 0.f;
+      if (n > 0) {
+        const uint32_t T_last = T - 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(int(T_last & 1)), int(T_last >> 1) & 1, abort_flag))) {
+          ok = false; break;
+        }
+        tc_fence_after();
+      }
 #pragma unroll 1
-        for (int q = 0; q < DH / 32; ++q) {
-          uint32_t ov[32];
+      for (int q = 0; q < DH / 32; ++q) {
+        uint32_t ov[32];
+        if (n > 0) {
           tmem_ld_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
           tmem_wait_ld();
+          if (q == DH / 32 - 1) {
+            // All of O is in registers: the next item's first P V may overwrite it.
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_o_free);
+          }
+        }
+        if (store_o) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
+          for (int e4 = 0; e4 < 4; ++e4) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w4[e] = have ? pack_bf16x2(__uint_as_float(ov[8 * e4 + 2 * e]) * inv_l,
+                                         __uint_as_float(ov[8 * e4 + 2 * e + 1]) * inv_l) : 0u;
+            reinterpret_cast<uint4*>(orow + q * 32)[e4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_p_full(b));
-      if (tr) LVA_TRACE_AT(7, t);
+      if (n > 0) ++nq;
+      if (store && hf == 0)
+        p.lse[plane * p.n_pad + grow] = have ? (m_ref + __log2f(l_row)) * 0.69314718055994530942f : -INFINITY;
     }
-
-    // ------------------------------------------------------------ epilogue
-    if (tr) LVA_TRACE_AT(16, 0);
-    if (ok && n > 0) {
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag))) ok = false;
-      else tc_fence_after();
-    }
-    if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 3); }
-    // Row sum over both halves.
-    const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
-    const int64_t grow = int64_t(i) * BN + row;           // row within the plane
-    const bool store = row < BN && grow < p.n_pad;
-    const bool have = ok && n > 0 && l_row > 0.f;
-    const float inv_l = have ? 1.f / l_row : 0.f;
-    // O row destination: tile order, or (fused inverse reorder) the row's raster position;
-    // padding rows have no raster position and are not written then.
-    __nv_bfloat16* orow;
-    bool store_o = store;
-    if (p.o_raster != nullptr) {
-      store_o = store && grow < p.n_valid;
-      const uint32_t raster = store_o ? tile_order_to_raster(uint32_t(grow), p.grid) : 0u;
-      orow = p.o_raster + (plane * p.n_valid + int64_t(raster)) * D + hf * DH;
-    } else {
-      orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
-    }
-#pragma unroll 1
-    for (int q = 0; q < DH / 32; ++q) {
-      uint32_t ov[32];
-      if (ok && n > 0) {
-        tmem_ld_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
-        tmem_wait_ld();
-      }
-      uint32_t w[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e)
-        w[e] = have ? pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l) : 0u;
-      if (store_o) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + q * 32);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-      }
-    }
-    if (tr) LVA_TRACE_AT(18, 0);
-    if (store && hf == 0)
-      p.lse[plane * p.n_pad + grow] = have ? (m_ref + __log2f(l_row)) * 0.69314718055994530942f : -INFINITY;
+    if (!ok) { *abort_flag = 1; if (lane == 0) report_fault(p.err, 5, 3); }
   }
 
   tc_fence_before();
@@ -521,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   }
 }
 
-template <int D, int BN>
+template <int D, int BN, int KPC>
 cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why) {
   using C = Cfg<D, BN>;
   const int64_t rows = int64_t(a.B) * a.H * a.n_pad;
@@ -544,7 +621,7 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, BN, KPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_BYTES);
     if (e != cudaSuccess) { *why = "cudaFuncSetAttribute(max dynamic smem) failed"; return e; }
     attr_set[dev] = true;
@@ -570,7 +647,9 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   p.err = a.err;
   const int64_t items = rows / a.block_size;
   if (items == 0) return cudaSuccess;
-  bsa_fwd_kernel<D, BN><<<dim3(unsigned(items)), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  p.items = items;
+  const int64_t grid = (items + KPC - 1) / KPC;
+  bsa_fwd_kernel<D, BN, KPC><<<dim3(unsigned(grid)), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -582,11 +661,26 @@ extern "C" int lva_trace_copy(void* dst, size_t bytes) {
 }
 #endif
 
+// Query blocks per CTA.  A CTA walks a run of consecutive query blocks: its prologue
+// (barriers, TMEM allocation, the first Q and K tiles) is paid once per run and the next
+// block's loads and first Q K^T overlap the current epilogue, while the hardware still hands
+// out runs in order as SMs free up.  That pays off for short CSR rows (a few key blocks per
+// query block) and costs tail balance and L2 locality for long ones.  With col_len taken as
+// the entry count: runs of 8 for rows averaging at most 3 key blocks, 4 for at most 8,
+// otherwise 1 (a capacity larger than the entry count therefore selects 1).
+template <int D, int BN>
+cudaError_t launch_dispatch(const AttnArgs& a, cudaStream_t stream, const char** why) {
+  const int64_t rows = int64_t(a.mask_heads) * (a.n_pad / a.block_size);
+  if (rows > 0 && a.col_len <= 3 * rows) return launch_cfg<D, BN, 8>(a, stream, why);
+  if (rows > 0 && a.col_len <= 8 * rows) return launch_cfg<D, BN, 4>(a, stream, why);
+  return launch_cfg<D, BN, 1>(a, stream, why);
+}
+
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why) {
-  if (a.d == 128 && a.block_size == 128) return launch_cfg<128, 128>(a, stream, why);
-  if (a.d == 128 && a.block_size == 64) return launch_cfg<128, 64>(a, stream, why);
-  if (a.d == 64 && a.block_size == 128) return launch_cfg<64, 128>(a, stream, why);
-  if (a.d == 64 && a.block_size == 64) return launch_cfg<64, 64>(a, stream, why);
+  if (a.d == 128 && a.block_size == 128) return launch_dispatch<128, 128>(a, stream, why);
+  if (a.d == 128 && a.block_size == 64) return launch_dispatch<128, 64>(a, stream, why);
+  if (a.d == 64 && a.block_size == 128) return launch_dispatch<64, 128>(a, stream, why);
+  if (a.d == 64 && a.block_size == 64) return launch_dispatch<64, 64>(a, stream, why);
   *why = "unsupported (d, block_size)";
   return cudaErrorInvalidValue;
 }

@@ -84,6 +84,7 @@ class VideoBlockSparseAttention:
         self.query_src = (torch.as_tensor(query_src, dtype=torch.int32).to(self.device).contiguous()
                           if query_src is not None else None)
         self._built_step = None
+        self.col_view = self.col_idx
 
     def build_mask(self, step: int = 0):
         """(Re)build the CSR; parametric window masks depend on the denoising step."""
@@ -94,6 +95,12 @@ class VideoBlockSparseAttention:
         self.params.step = key
         lb.lva_build_block_mask(self.params, self.dense_mask, self.row_ptr, self.col_idx, self.nnz)
         self._built_step = key
+        # A mask built once can tell the attention call its exact entry count (read back once);
+        # short rows then get CTAs that walk several query blocks.  Per-step masks keep the
+        # capacity, so no step waits for a device-to-host read.
+        self.col_view = self.col_idx
+        if not steps_matter:
+            self.col_view = self.col_idx[:max(1, int(self.nnz.item()))]
 
     @staticmethod
     def _stacked(q, k, v):
@@ -125,7 +132,7 @@ class VideoBlockSparseAttention:
 
     def attend(self):
         lb.lva_block_sparse_attn(self.q_t, self.k_t, self.v_t, self.o_t, self.lse, self.n_valid,
-                                 self.block_size, self.row_ptr, self.col_idx, self.mask_heads, self.scale,
+                                 self.block_size, self.row_ptr, self.col_view, self.mask_heads, self.scale,
                                  self.query_src)
         if self.query_src is not None:
             lb.lva_broadcast_blocks(self.o_t, self.lse, self.block_size, self.query_src)
@@ -134,7 +141,7 @@ class VideoBlockSparseAttention:
         """Attention with the inverse reorder fused into its epilogue: O goes straight to
         raster order (``self.o``); LSE stays in tile order (``self.lse``)."""
         lb.lva_block_sparse_attn_raster(self.q_t, self.k_t, self.v_t, self.o, self.lse, self.n_valid,
-                                        self.block_size, self.row_ptr, self.col_idx, self.mask_heads,
+                                        self.block_size, self.row_ptr, self.col_view, self.mask_heads,
                                         self.scale, self.grid, self.tile)
 
     def reorder_out(self):
@@ -209,12 +216,12 @@ class VideoBlockSparseAttention:
             qkv_t = (self.q_t[b:b + 1, h0:h1], self.k_t[b:b + 1, h0:h1], self.v_t[b:b + 1, h0:h1])
             if self.query_src is None:
                 lb.lva_block_sparse_attn_raster(*qkv_t, self.o[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], N,
-                                                self.block_size, row_ptr, self.col_idx, 1 if mh == 1 else hn,
+                                                self.block_size, row_ptr, self.col_view, 1 if mh == 1 else hn,
                                                 self.scale, self.grid, self.tile)
             else:
                 qs = self.query_src if self.query_src.shape[0] == 1 else self.query_src[h0:h1]
                 lb.lva_block_sparse_attn(*qkv_t, self.o_t[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], N,
-                                         self.block_size, row_ptr, self.col_idx, 1 if mh == 1 else hn,
+                                         self.block_size, row_ptr, self.col_view, 1 if mh == 1 else hn,
                                          self.scale, qs)
                 lb.lva_broadcast_blocks(self.o_t[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], self.block_size, qs)
                 lb.lva_reorder_tokens(self.o_t[b, h0:h1].reshape(P, self.n_pad, d),
@@ -272,7 +279,8 @@ class SquadTwoPass:
             col_idx = torch.empty(lb.lva_block_mask_max_nnz(p), dtype=torch.int32, **kw)
             nnz = torch.empty(1, dtype=torch.int32, **kw)
             lb.lva_build_block_mask(p, None, row_ptr, col_idx, nnz)
-            self.csr[name] = (row_ptr, col_idx)
+            # exact entry counts (read once): rows of 2-4 blocks get multi-block CTAs
+            self.csr[name] = (row_ptr, col_idx[:max(1, int(nnz.item()))])
 
     def __call__(self, q, k, v):
         rp, ci = self.csr["local"]

@@ -167,7 +167,10 @@ lva_status lva_build_block_mask(const lva_mask_params* params, const uint8_t* de
  * q, k, v, o: device bf16 [B, H, n_pad, d], 16-byte aligned.  lse: device fp32 [B, H, n_pad].
  * row_ptr: device [mask_heads*nb + 1]; col_idx: device, col_len entries (the kernel never
  * reads past col_len; CSR entries out of range are skipped and reported through
- * lva_device_error as LVA_ERR_INVALID_ARG).
+ * lva_device_error as LVA_ERR_INVALID_ARG).  col_len may be the capacity of col_idx or the
+ * exact entry count; the exact count lets the call see short rows, for which each CTA then
+ * processes a run of consecutive query blocks (8 when rows average at most 3 key blocks, 4
+ * when at most 8; results are identical either way).
  * query_src: NULL, or device int32 [src_heads, nb] (src_heads in {1, H}): query blocks with
  * query_src[h_s*nb + i] != i are not computed here (their O/LSE are left untouched for
  * lva_broadcast_blocks to fill).

@@ -249,3 +249,49 @@ def test_fused_raster_output_matches_separate_reorder(name, grid, tile, d, bs):
     from tests.gpu_helpers import bits
     assert np.array_equal(bits(layer.o), bits(o_sep))
     assert np.array_equal(bits(layer.lse), bits(lse_sep))
+
+
+@pytest.mark.parametrize("d,bs,hm,with_src", [(128, 128, 1, False), (128, 128, 3, True), (64, 64, 3, False)])
+def test_multi_block_ctas_match_single_block_ctas(d, bs, hm, with_src):
+    """Short rows passed with their exact entry count run CTAs that walk 4 query blocks each;
+    the same CSR passed with a larger capacity runs one query block per CTA.  Same rows, same
+    arithmetic: the outputs must agree bit for bit (including empty rows and skipped blocks)."""
+    import block_sparse_attention_lva_b200 as lva
+    from tests.gpu_helpers import bits
+    dev = require_gpu()
+    B, H = 1, 3
+    n_pad = 64 * bs
+    n_valid = n_pad - 37                                     # a ragged tail
+    nb = n_pad // bs
+    q, k, v = (_rand_bf16((B, H, n_pad, d), s) for s in (11, 12, 13))
+    rng = np.random.default_rng(d + bs + hm)
+    masks = rng.random((hm, nb, nb)) < 0.04                  # ~2.6 key blocks per row
+    masks[0, 5] = False                                      # an empty row
+    rp, ci = dense_to_csr(masks)
+    row_ptr = torch.from_numpy(rp).to(dev)
+    exact = torch.from_numpy(ci).to(dev)
+    padded = torch.zeros(hm * nb * nb, dtype=torch.int32, device=dev)
+    padded[:ci.size] = exact
+    src = None
+    if with_src:
+        s_ = np.tile(np.arange(nb, dtype=np.int32), (H, 1))
+        s_[1, 1::2] = np.arange(0, nb, 2, dtype=np.int32)   # head 1: odd blocks copy the even one before
+        src = torch.from_numpy(s_).to(dev)
+    outs = []
+    for col in (exact, padded):
+        o = torch.full((B, H, n_pad, d), float("nan"), dtype=torch.bfloat16, device=dev)
+        lse = torch.full((B, H, n_pad), float("nan"), dtype=torch.float32, device=dev)
+        lva.lva_block_sparse_attn(q.to(dev), k.to(dev), v.to(dev), o, lse, n_valid, bs, row_ptr, col, hm,
+                                  d ** -0.5, src)
+        torch.cuda.synchronize()
+        assert lva.lva_device_error() == (0, 0)
+        outs.append((o, lse))
+    assert np.array_equal(bits(outs[0][0]), bits(outs[1][0]))
+    assert np.array_equal(bits(outs[0][1]), bits(outs[1][1]))
+    # and against the oracle for the computed blocks
+    o_ref, lse_ref = attention_blocked(q, k, v, masks, bs, n_valid, d ** -0.5)
+    computed = np.ones((H, nb), bool) if src is None else (src.cpu().numpy() == np.arange(nb))
+    for h in range(H):
+        rows = np.concatenate([np.arange(i * bs, (i + 1) * bs) for i in range(nb) if computed[h, i]])
+        check_o_lse(outs[0][0][:, h:h + 1, rows], outs[0][1][:, h:h + 1, rows], o_ref[:, h:h + 1, rows],
+                    lse_ref[:, h:h + 1, rows], f"head {h}")
