@@ -174,9 +174,13 @@ class VideoBlockSparseAttention:
         ordered after the last copy back (synchronise that stream before reading o_host).
         """
         B, H, N, d = self.B, self.H, self.n_valid, self.d
-        assert tuple(qkv_host.shape) == (3, B, H, N, d) and qkv_host.is_pinned()
-        assert tuple(o_host.shape) == (B, H, N, d) and o_host.is_pinned()
-        assert tuple(lse_host.shape) == (B, H, self.n_pad) and lse_host.is_pinned()
+        for name, t, shape, dtype in (("qkv_host", qkv_host, (3, B, H, N, d), torch.bfloat16),
+                                      ("o_host", o_host, (B, H, N, d), torch.bfloat16),
+                                      ("lse_host", lse_host, (B, H, self.n_pad), torch.float32)):
+            if tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {shape}")
+            if not t.is_pinned():
+                raise ValueError(f"{name} must be in pinned host memory (copies overlap compute)")
         if not hasattr(self, "_host_io"):
             self._host_io = dict(
                 qkv_dev=torch.empty((3, B, H, N, d), dtype=torch.bfloat16, device=self.device),
