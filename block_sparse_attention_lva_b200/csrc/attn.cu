@@ -1,11 +1,14 @@
 // attn.cu -- block-sparse FlashAttention-style forward for sm_100a (TMA + tcgen05 + TMEM).
 //
-// One CTA computes one (batch, head, query block i): it walks only the key blocks listed
-// in CSR row (h_m, i) -- the precomputed skip list of the CalibAtt page ("Accelerating
-// Text-to-Video Generation with Calibrated Sparse Attention", section 2 B) or the LVSA
-// window + anchor set ("LVSA: Training-Free Sparse Attention for Long Video Diffusion",
-// technical summary section 2) -- with an online softmax, so the cost is proportional to
-// the number of listed blocks.
+// A CTA computes a run of consecutive (batch, head, query block i) items -- one, or 4 or 8
+// when the CSR rows are short -- and for each walks only the key blocks listed in CSR row
+// (h_m, i): the precomputed skip list of the CalibAtt page ("Accelerating Text-to-Video
+// Generation with Calibrated Sparse Attention", section 2 B) or the LVSA window + anchor set
+// ("LVSA: Training-Free Sparse Attention for Long Video Diffusion", technical summary
+// section 2), with an online softmax, so the cost is proportional to the number of listed
+// blocks.  O goes to tile order, or straight to raster order (the inverse token reorder
+// fused into the epilogue); Q/K/V rows come from plane-major 2D tensor maps, or from 3D
+// maps that gather the window-transposed order in place (the SQuad page's global pass).
 //
 // Pipeline: S and P are double-buffered in TMEM (S_0, S_1, P_0, P_1, O = 512 columns), so
 // the MMA issuer computes S(t+2) = Q K_{t+2}^T as soon as the softmax has read S(t), and
