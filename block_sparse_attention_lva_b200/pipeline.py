@@ -162,7 +162,7 @@ class VideoBlockSparseAttention:
         return self.o, self.lse
 
 
-    def forward_host(self, qkv_host, o_host, lse_host, step: int = 0, chunks: int = 6):
+    def forward_host(self, qkv_host, o_host, lse_host, step: int = 0, chunks: int = 6, wait: bool = True):
         """One layer step from and to pinned host memory, with the copies overlapped.
 
         ``qkv_host``: pinned bf16 [3, B, H, N, d] (raster Q, K, V); ``o_host``: pinned bf16
@@ -170,8 +170,14 @@ class VideoBlockSparseAttention:
         LSE, written).  Heads are independent given the mask, so the step runs per group of
         heads of one batch element: the host-to-device copy of group c+1 and the
         device-to-host copy of group c-1 proceed while group c is reordered and attended.
-        Copies use their own streams; the call returns with the caller's current stream
-        ordered after the last copy back (synchronise that stream before reading o_host).
+        Consecutive calls overlap too: the device staging and output buffers are
+        double-buffered, so a call's host-to-device copies start while the previous call is
+        still computing and copying back.
+
+        Returns a CUDA event that completes when ``o_host`` and ``lse_host`` hold this step's
+        results; the host buffers must not be rewritten or read before then.  With ``wait``
+        the caller's current stream is also ordered after it (synchronise that stream before
+        reading the results on the host).
         """
         B, H, N, d = self.B, self.H, self.n_valid, self.d
         for name, t, shape, dtype in (("qkv_host", qkv_host, (3, B, H, N, d), torch.bfloat16),
@@ -182,21 +188,27 @@ class VideoBlockSparseAttention:
             if not t.is_pinned():
                 raise ValueError(f"{name} must be in pinned host memory (copies overlap compute)")
         if not hasattr(self, "_host_io"):
+            mk = lambda shape, dt: torch.empty(shape, dtype=dt, device=self.device)
             self._host_io = dict(
-                qkv_dev=torch.empty((3, B, H, N, d), dtype=torch.bfloat16, device=self.device),
+                qkv=[mk((3, B, H, N, d), torch.bfloat16) for _ in range(2)],
+                o=[mk((B, H, N, d), torch.bfloat16) for _ in range(2)],
+                lse=[mk((B, H, self.n_pad), torch.float32) for _ in range(2)],
+                staging_free=[None, None], out_free=[None, None], slot=0,
                 h2d=torch.cuda.Stream(self.device), d2h=torch.cuda.Stream(self.device))
         io = self._host_io
-        qkv_dev, s_h2d, s_d2h = io["qkv_dev"], io["h2d"], io["d2h"]
+        sl = io["slot"]
+        io["slot"] = sl ^ 1
+        qkv_dev, o_dev, lse_dev = io["qkv"][sl], io["o"][sl], io["lse"][sl]
+        s_h2d, s_d2h = io["h2d"], io["d2h"]
         cur = torch.cuda.current_stream(self.device)
         groups = []
         per = max(1, -(-H // max(1, chunks // max(1, B))))
         for b in range(B):
             for h0 in range(0, H, per):
                 groups.append((b, h0, min(H, h0 + per)))
-        # Ordering: copies into the staging buffer wait for the previous step's compute.
-        s_h2d.wait_stream(cur)
-        s_d2h.wait_stream(cur)
-        self.build_mask(step)
+        # Host-to-device: staging slot `sl` was last read by the compute of two calls ago.
+        if io["staging_free"][sl] is not None:
+            s_h2d.wait_event(io["staging_free"][sl])
         in_ready, out_ready = [], []
         for b, h0, h1 in groups:
             with torch.cuda.stream(s_h2d):
@@ -205,6 +217,10 @@ class VideoBlockSparseAttention:
                 ev = torch.cuda.Event()
                 ev.record(s_h2d)
             in_ready.append(ev)
+        self.build_mask(step)
+        # Output slot `sl` was last read by the copies back of two calls ago.
+        if io["out_free"][sl] is not None:
+            cur.wait_event(io["out_free"][sl])
         # The static-mask and repetitive-head tables are indexed per head of the group.
         nb = self.nb
         for (b, h0, h1), ev in zip(groups, in_ready):
@@ -219,28 +235,35 @@ class VideoBlockSparseAttention:
             row_ptr = self.row_ptr if mh == 1 else self.row_ptr[h0 * nb:]
             qkv_t = (self.q_t[b:b + 1, h0:h1], self.k_t[b:b + 1, h0:h1], self.v_t[b:b + 1, h0:h1])
             if self.query_src is None:
-                lb.lva_block_sparse_attn_raster(*qkv_t, self.o[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], N,
+                lb.lva_block_sparse_attn_raster(*qkv_t, o_dev[b:b + 1, h0:h1], lse_dev[b:b + 1, h0:h1], N,
                                                 self.block_size, row_ptr, self.col_view, 1 if mh == 1 else hn,
                                                 self.scale, self.grid, self.tile)
             else:
                 qs = self.query_src if self.query_src.shape[0] == 1 else self.query_src[h0:h1]
-                lb.lva_block_sparse_attn(*qkv_t, self.o_t[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], N,
+                lb.lva_block_sparse_attn(*qkv_t, self.o_t[b:b + 1, h0:h1], lse_dev[b:b + 1, h0:h1], N,
                                          self.block_size, row_ptr, self.col_view, 1 if mh == 1 else hn,
                                          self.scale, qs)
-                lb.lva_broadcast_blocks(self.o_t[b:b + 1, h0:h1], self.lse[b:b + 1, h0:h1], self.block_size, qs)
+                lb.lva_broadcast_blocks(self.o_t[b:b + 1, h0:h1], lse_dev[b:b + 1, h0:h1], self.block_size, qs)
                 lb.lva_reorder_tokens(self.o_t[b, h0:h1].reshape(P, self.n_pad, d),
-                                      self.o[b, h0:h1].reshape(P, N, d), self.grid, self.tile, self.n_pad,
+                                      o_dev[b, h0:h1].reshape(P, N, d), self.grid, self.tile, self.n_pad,
                                       inverse=True)
             ev = torch.cuda.Event()
             ev.record(cur)
             out_ready.append(ev)
+        staging_free = torch.cuda.Event()
+        staging_free.record(cur)
+        io["staging_free"][sl] = staging_free
         for (b, h0, h1), ev in zip(groups, out_ready):
             s_d2h.wait_event(ev)
             with torch.cuda.stream(s_d2h):
-                o_host[b, h0:h1].copy_(self.o[b, h0:h1], non_blocking=True)
-                lse_host[b, h0:h1].copy_(self.lse[b, h0:h1], non_blocking=True)
-        cur.wait_stream(s_d2h)
-        return o_host, lse_host
+                o_host[b, h0:h1].copy_(o_dev[b, h0:h1], non_blocking=True)
+                lse_host[b, h0:h1].copy_(lse_dev[b, h0:h1], non_blocking=True)
+        done = torch.cuda.Event()
+        done.record(s_d2h)
+        io["out_free"][sl] = done
+        if wait:
+            cur.wait_event(done)
+        return done
 
 
 class SquadTwoPass:
