@@ -298,7 +298,9 @@ def lva_aggregate_masks(masks, out, rho: float):
     """Blocks kept by at least a fraction ``rho`` of the prompt masks ``masks[P, ...]``."""
     import torch
     _cuda_tensor(masks, "masks", torch.uint8)
-    _cuda_tensor(out, "out", torch.uint8, masks[0].numel())
+    _cuda_tensor(out, "out", torch.uint8)
+    _need(masks.dim() >= 1 and masks.shape[0] >= 1 and out.numel() == masks[0].numel(),
+          "out must have as many elements as one prompt's mask masks[p]")
     _check(lib.lva_aggregate_masks(_ptr(masks), _ptr(out), masks.shape[0], out.numel(), ctypes.c_double(rho),
                                    ctypes.c_void_p(_stream(masks.device))))
     return out

@@ -32,10 +32,10 @@ lva_status from_cuda(cudaError_t e, const char* what) {
 }
 
 // Kernel-side error word: [0] = status, [1] = detail.  One copy per device (module global);
-// its device address is looked up once per device.
+// its device address is looked up once per device (on every call past the cache).
 __device__ int g_device_error[2];
 
-int* g_err_ptr[128] = {};
+std::atomic<int*> g_err_ptr[kMaxCachedDevices] = {};
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -43,13 +43,16 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 int* device_error_word() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
-  if (g_err_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    g_err_ptr[dev] = static_cast<int*>(p);
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  const bool cacheable = dev >= 0 && dev < kMaxCachedDevices;
+  if (cacheable) {
+    int* cached = g_err_ptr[dev].load(std::memory_order_acquire);
+    if (cached != nullptr) return cached;
   }
-  return g_err_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  if (cacheable) g_err_ptr[dev].store(static_cast<int*>(p), std::memory_order_release);
+  return static_cast<int*>(p);
 }
 
 }  // namespace lva

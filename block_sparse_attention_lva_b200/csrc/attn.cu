@@ -620,15 +620,12 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
     *why = "cuTensorMapEncodeTiled failed or is unavailable";
     return cudaErrorInvalidValue;
   }
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(bsa_fwd_kernel<D, BN, KPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM_BYTES);
-    if (e != cudaSuccess) { *why = "cudaFuncSetAttribute(max dynamic smem) failed"; return e; }
-    attr_set[dev] = true;
-  }
+  static DeviceFlags attr_set = {};
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(bsa_fwd_kernel<D, BN, KPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_BYTES);
+  });
+  if (e != cudaSuccess) { *why = "cudaFuncSetAttribute(max dynamic smem) failed"; return e; }
   AttnParams p;
   p.H = a.H;
   p.nb = int(a.n_pad / a.block_size);

@@ -103,13 +103,17 @@ __global__ void aggregate_kernel(const uint8_t* __restrict__ masks, uint8_t* __r
 }
 
 int sm_count() {
-  static int cached[64] = {};
+  static std::atomic<int> cached[kMaxCachedDevices] = {};
   int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && cached[dev]) return cached[dev];
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const bool cacheable = dev >= 0 && dev < kMaxCachedDevices;
+  if (cacheable) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  if (dev < 64) cached[dev] = n;
+  if (cacheable) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -120,15 +124,12 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   int p2 = 1;
   while (p2 < a.nb) p2 <<= 1;
   const size_t smem = size_t(p2) * 8 + size_t(a.nb + 1) * 8;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
+  static DeviceFlags attr_set = {};
+  cudaError_t e = once_per_device(attr_set, [] {
     const int max_smem = (kSelectMaxBlocks + kSelectMaxBlocks + 1) * 8;
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
+    return cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+  });
+  if (e != cudaSuccess) return e;
   const int64_t grid = a.rows < int64_t(sm_count()) * 8 ? a.rows : int64_t(sm_count()) * 8;
   select_kernel<<<unsigned(grid), kSelThreads, smem, stream>>>(a.energy, a.mask, a.rows, a.nb, p2,
                                                                a.eps, a.err);

@@ -306,15 +306,12 @@ cudaError_t launch_energy_cfg(const EnergyArgs& a, cudaStream_t stream, const ch
     *why = "cuTensorMapEncodeTiled failed or is unavailable";
     return cudaErrorInvalidValue;
   }
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(block_energy_kernel<D, BN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) { *why = "cudaFuncSetAttribute(max dynamic smem) failed"; return e; }
-    attr_set[dev] = true;
-  }
+  static DeviceFlags attr_set = {};
+  cudaError_t e = once_per_device(attr_set, [] {
+    return cudaFuncSetAttribute(block_energy_kernel<D, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                C::SMEM_BYTES);
+  });
+  if (e != cudaSuccess) { *why = "cudaFuncSetAttribute(max dynamic smem) failed"; return e; }
   EnergyParams p;
   p.H = a.H;
   p.nb = int(a.n_pad / a.block_size);

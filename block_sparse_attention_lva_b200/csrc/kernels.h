@@ -3,11 +3,31 @@
 // launcher returns the cudaError_t of its launch(es).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace lva {
+
+// Per-device setup done once (a kernel's shared-memory limit, a looked-up attribute).  The
+// flags are atomic so that concurrent host threads are safe; the setup itself must be
+// idempotent, since two threads may both run it before either sets the flag.  Devices past
+// the cache run the setup on every call.
+constexpr int kMaxCachedDevices = 64;
+using DeviceFlags = std::atomic<bool>[kMaxCachedDevices];
+
+template <class F>
+cudaError_t once_per_device(DeviceFlags& done, F&& setup) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < kMaxCachedDevices;
+  if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = setup();
+  if (e == cudaSuccess && cached) done[dev].store(true, std::memory_order_release);
+  return e;
+}
 
 struct ReorderArgs {
   const void* src;

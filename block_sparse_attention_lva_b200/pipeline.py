@@ -63,6 +63,9 @@ class VideoBlockSparseAttention:
             if static_mask is None:
                 raise ValueError("static mask kind needs static_mask")
             sm = torch.as_tensor(static_mask, dtype=torch.uint8)
+            if sm.dim() != 3 or sm.shape[0] not in (1, H) or tuple(sm.shape[1:]) != (self.nb, self.nb):
+                raise ValueError(f"static_mask must have shape [1 or {H}, {self.nb}, {self.nb}], "
+                                 f"got {tuple(sm.shape)}")
             self.mask_heads = sm.shape[0]
             self.dense_mask = sm.to(self.device).contiguous()
         self.params = mask_params_for(self.mask, self.n_pad, self.n_valid, block_size, self.mask_heads)
@@ -83,6 +86,9 @@ class VideoBlockSparseAttention:
         self.nnz = torch.empty(1, dtype=torch.int32, **kw)
         self.query_src = (torch.as_tensor(query_src, dtype=torch.int32).to(self.device).contiguous()
                           if query_src is not None else None)
+        if self.query_src is not None and (self.query_src.dim() != 2 or self.query_src.shape[0] not in (1, H)
+                                           or self.query_src.shape[1] != self.nb):
+            raise ValueError(f"query_src must have shape [1 or {H}, {self.nb}]")
         self._built_step = None
         self.col_view = self.col_idx
 
@@ -193,7 +199,7 @@ class VideoBlockSparseAttention:
                 qkv=[mk((3, B, H, N, d), torch.bfloat16) for _ in range(2)],
                 o=[mk((B, H, N, d), torch.bfloat16) for _ in range(2)],
                 lse=[mk((B, H, self.n_pad), torch.float32) for _ in range(2)],
-                staging_free=[None, None], out_free=[None, None], slot=0,
+                staging_free=[None, None], out_free=[None, None], computed=None, slot=0,
                 h2d=torch.cuda.Stream(self.device), d2h=torch.cuda.Stream(self.device))
         io = self._host_io
         sl = io["slot"]
@@ -217,10 +223,14 @@ class VideoBlockSparseAttention:
                 ev = torch.cuda.Event()
                 ev.record(s_h2d)
             in_ready.append(ev)
-        self.build_mask(step)
-        # Output slot `sl` was last read by the copies back of two calls ago.
+        # Output slot `sl` was last read by the copies back of two calls ago; the tile-order
+        # buffers and the CSR are shared by all calls, so the mask build and the compute also
+        # follow the previous call's compute (a no-op when the caller keeps one stream).
         if io["out_free"][sl] is not None:
             cur.wait_event(io["out_free"][sl])
+        if io["computed"] is not None:
+            cur.wait_event(io["computed"])
+        self.build_mask(step)
         # The static-mask and repetitive-head tables are indexed per head of the group.
         nb = self.nb
         for (b, h0, h1), ev in zip(groups, in_ready):
@@ -253,6 +263,7 @@ class VideoBlockSparseAttention:
         staging_free = torch.cuda.Event()
         staging_free.record(cur)
         io["staging_free"][sl] = staging_free
+        io["computed"] = staging_free
         for (b, h0, h1), ev in zip(groups, out_ready):
             s_d2h.wait_event(ev)
             with torch.cuda.stream(s_d2h):

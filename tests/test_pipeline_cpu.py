@@ -16,3 +16,23 @@ def test_stacked_detection_needs_one_storage():
     a, b, c = flat[:256].view(1, 2, 16, 8), flat[256:512].view(1, 2, 16, 8), flat[512:].view(1, 2, 16, 8)
     assert VideoBlockSparseAttention._stacked(a, b, c)
     assert not VideoBlockSparseAttention._stacked(a, b.view(2, 1, 16, 8), c)
+
+
+def test_layer_rejects_misshapen_static_mask_and_query_src():
+    import pytest
+    # grid 2x8x8 = 128 tokens in 64-token blocks: nb = 2
+    kw = dict(B=1, H=3, d=64, grid=(2, 8, 8), tile=(1, 4, 4), block_size=64, device="cpu")
+    with pytest.raises(ValueError, match="static_mask"):
+        VideoBlockSparseAttention(mask={"kind": "static"}, static_mask=torch.ones(2, 2, 2, dtype=torch.uint8), **kw)
+    with pytest.raises(ValueError, match="static_mask"):
+        VideoBlockSparseAttention(mask={"kind": "static"}, static_mask=torch.ones(3, 2, 3, dtype=torch.uint8), **kw)
+    with pytest.raises(ValueError, match="static_mask"):
+        VideoBlockSparseAttention(mask={"kind": "static"}, static_mask=torch.ones(12, dtype=torch.uint8), **kw)
+    layer = VideoBlockSparseAttention(mask={"kind": "static"}, static_mask=torch.ones(3, 2, 2, dtype=torch.uint8), **kw)
+    assert layer.mask_heads == 3
+    win = {"kind": "window_anchor", "unit": 64, "radius": 1, "anchors": 0}
+    with pytest.raises(ValueError, match="query_src"):
+        VideoBlockSparseAttention(mask=win, query_src=torch.zeros(2, 2, dtype=torch.int32), **kw)
+    with pytest.raises(ValueError, match="query_src"):
+        VideoBlockSparseAttention(mask=win, query_src=torch.zeros(1, 3, dtype=torch.int32), **kw)
+    VideoBlockSparseAttention(mask=win, query_src=torch.zeros(1, 2, dtype=torch.int32), **kw)
