@@ -58,6 +58,7 @@ SIGNATURES = {
     "lva_select_blocks": (_c_int, [_vp, _vp, _c_i64, _c_int, ctypes.c_double, _vp]),
     "lva_aggregate_masks": (_c_int, [_vp, _vp, _c_int, _c_i64, ctypes.c_double, _vp]),
     "lva_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
+    "lva_selftest_wait": (_c_int, [_c_int, _vp]),
 }
 
 
@@ -312,3 +313,10 @@ def lva_device_error(stream=None):
     s = _stream() if stream is None else stream
     _check(lib.lva_device_error(ctypes.c_void_p(s), ctypes.byref(st), ctypes.byref(det)))
     return st.value, det.value
+
+
+def lva_selftest_wait(mode: int, stream=None):
+    """Runs the bounded-wait self-test kernel (mode 0: runs out, 1: aborted, 2: completes) on
+    the current stream; read the outcome with ``lva_device_error``."""
+    s = _stream() if stream is None else stream
+    _check(lib.lva_selftest_wait(int(mode), ctypes.c_void_p(s)))

@@ -342,6 +342,13 @@ lva_status lva_aggregate_masks(const uint8_t* masks, uint8_t* out, int prompts, 
   return from_cuda(launch_aggregate(a, stream), "aggregate launch");
 }
 
+lva_status lva_selftest_wait(int mode, cudaStream_t stream) {
+  if (mode < 0 || mode > 2) return fail(LVA_ERR_INVALID_ARG, "selftest_wait: mode must be 0, 1 or 2");
+  int* err = device_error_word();
+  if (err == nullptr) return fail(LVA_ERR_CUDA, "selftest_wait: cannot locate the device error word");
+  return from_cuda(launch_wait_selftest(mode, err, stream), "selftest_wait launch");
+}
+
 lva_status lva_device_error(cudaStream_t stream, lva_status* status, int* detail) {
   if (status == nullptr) return fail(LVA_ERR_INVALID_ARG, "device_error: null status");
   int* err = device_error_word();

@@ -143,4 +143,8 @@ bool make_window_gather_map(CUtensorMap* m, const void* base, int64_t planes, in
 // Device error word of the current device (from api.cu).
 int* device_error_word();
 
+// Bounded-wait self-test (selftest.cu): mode 0 = nothing arrives, 1 = abort flag raised,
+// 2 = the peer arrives.
+cudaError_t launch_wait_selftest(int mode, int* err, cudaStream_t stream);
+
 }  // namespace lva

@@ -323,6 +323,23 @@ lva_status lva_aggregate_masks(const uint8_t* masks, uint8_t* out, int prompts, 
  */
 lva_status lva_device_error(cudaStream_t stream, lva_status* status, int* detail);
 
+/*
+ * lva_selftest_wait -- diagnostic of the kernels' bounded waits; the pages have no counterpart.
+ *
+ * Every pipeline wait in these kernels (TMA arrivals, MMA completions, softmax hand-offs)
+ * polls its mbarrier for at most 2 s of device wall time (%globaltimer), or until another role
+ * of the same CTA raises the CTA's abort flag, then gives up and records LVA_ERR_TIMEOUT in
+ * the device error word, so a broken pipeline ends with a status instead of a hung GPU.  This
+ * call runs that same wait in a one-CTA kernel on `stream`:
+ *   mode 0: nothing arrives; after about 2 s the error word holds (LVA_ERR_TIMEOUT, 100);
+ *   mode 1: a second warp raises the abort flag after about 1 ms;
+ *           the error word holds (LVA_ERR_TIMEOUT, 101);
+ *   mode 2: a second warp arrives after about 1 ms; the wait completes, nothing is recorded.
+ * Read the outcome with lva_device_error.  The kernel touches no caller memory; the context
+ * stays usable in every mode.  Returns LVA_ERR_INVALID_ARG for another mode.
+ */
+lva_status lva_selftest_wait(int mode, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

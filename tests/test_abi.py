@@ -128,3 +128,9 @@ def test_window_transposed_attn_argument_checks():
     assert call(32768, 256, d=96) == 2      # unsupported head dim
     assert lib.lva_window_transposed_attn(vp, vp, vp, None, vp, 1, 2, 32768, 128, 256, 128, vp, vp, 4, 1,
                                           ctypes.c_float(0.1), None) == 1
+
+
+def test_selftest_wait_rejects_unknown_mode():
+    from block_sparse_attention_lva_b200._binding import lib
+    assert lib.lva_selftest_wait(3, None) == 1
+    assert lib.lva_selftest_wait(-1, None) == 1
