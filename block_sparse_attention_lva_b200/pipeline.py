@@ -186,11 +186,13 @@ class VideoBlockSparseAttention:
         reading the results on the host).
         """
         B, H, N, d = self.B, self.H, self.n_valid, self.d
-        for name, t, shape, dtype in (("qkv_host", qkv_host, (3, B, H, N, d), torch.bfloat16),
-                                      ("o_host", o_host, (B, H, N, d), torch.bfloat16),
-                                      ("lse_host", lse_host, (B, H, self.n_pad), torch.float32)):
+        bufs = (("qkv_host", qkv_host, (3, B, H, N, d), torch.bfloat16),
+                ("o_host", o_host, (B, H, N, d), torch.bfloat16),
+                ("lse_host", lse_host, (B, H, self.n_pad), torch.float32))
+        for name, t, shape, dtype in bufs:
             if tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous():
                 raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {shape}")
+        for name, t, _, _ in bufs:
             if not t.is_pinned():
                 raise ValueError(f"{name} must be in pinned host memory (copies overlap compute)")
         if not hasattr(self, "_host_io"):

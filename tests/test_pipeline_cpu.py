@@ -36,3 +36,22 @@ def test_layer_rejects_misshapen_static_mask_and_query_src():
     with pytest.raises(ValueError, match="query_src"):
         VideoBlockSparseAttention(mask=win, query_src=torch.zeros(1, 3, dtype=torch.int32), **kw)
     VideoBlockSparseAttention(mask=win, query_src=torch.zeros(1, 2, dtype=torch.int32), **kw)
+
+
+def test_host_step_rejects_bad_buffers_before_any_copy():
+    import pytest
+    kw = dict(B=1, H=2, d=64, grid=(2, 8, 8), tile=(1, 4, 4), block_size=64, device="cpu")
+    layer = VideoBlockSparseAttention(mask={"kind": "all"}, **kw)
+    N, n_pad = 128, 128
+    qkv = torch.zeros((3, 1, 2, N, 64), dtype=torch.bfloat16)
+    o = torch.zeros((1, 2, N, 64), dtype=torch.bfloat16)
+    lse = torch.zeros((1, 2, n_pad), dtype=torch.float32)
+    with pytest.raises(ValueError, match="qkv_host"):
+        layer.forward_host(qkv[:, :, :1], o, lse)                        # wrong head count
+    with pytest.raises(ValueError, match="o_host"):
+        layer.forward_host(qkv, o.float(), lse)                          # wrong dtype
+    with pytest.raises(ValueError, match="lse_host"):
+        layer.forward_host(qkv, o, torch.zeros((1, 2, n_pad, 2))[..., 0])  # not contiguous
+    with pytest.raises(ValueError, match="pinned"):
+        layer.forward_host(qkv, o, lse)                                  # pageable host memory
+    assert not hasattr(layer, "_host_io")                                # nothing was allocated
