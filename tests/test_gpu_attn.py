@@ -50,6 +50,7 @@ def _attn_gpu(q, k, v, masks, bs, n_valid, scale):
     (1, 1, 512, 512, 64, 64, 1, 1.0, 4),
     (1, 2, 4096, 4096, 128, 128, 2, 1.0, 5),
     (1, 1, 384, 1, 128, 128, 1, 1.0, 6),
+    (1, 2, 256, 0, 128, 128, 1, 1.0, 7),     # every key is padding: all rows empty
 ])
 def test_against_oracle_full(B, H, n_pad, n_valid, d, bs, hm, density, seed):
     q = _rand_bf16((B, H, n_pad, d), seed)
@@ -66,6 +67,17 @@ def test_against_oracle_full(B, H, n_pad, n_valid, d, bs, hm, density, seed):
     o, lse = _attn_gpu(q, k, v, masks, bs, n_valid, scale)
     o_ref, lse_ref = attention_blocked(q, k, v, masks, bs, n_valid, scale)
     check_o_lse(o, lse, o_ref, lse_ref, f"shape {(B, H, n_pad, d, bs)}")
+
+
+@pytest.mark.parametrize("d,bs", [(128, 128), (64, 64)])
+def test_all_rows_empty(d, bs):
+    """An empty CSR (no entries at all): every row gives O = 0 and LSE = -inf."""
+    B, H, n_pad = 2, 3, 1024
+    q, k, v = (_rand_bf16((B, H, n_pad, d), 70 + t) for t in range(3))
+    masks = np.zeros((H, n_pad // bs, n_pad // bs), dtype=bool)
+    o, lse = _attn_gpu(q, k, v, masks, bs, n_pad - 5, 1.0 / math.sqrt(d))
+    assert torch.count_nonzero(o.float().cpu()).item() == 0
+    assert bool(torch.all(lse.cpu() == float("-inf")))
 
 
 def test_many_items_mixed_rows():
