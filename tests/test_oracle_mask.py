@@ -61,6 +61,26 @@ def test_frame_window_count_small(step):
         assert total == 10375 and min(lengths) == 28 and max(lengths) == 53
 
 
+def test_padding_only_blocks_take_the_last_real_unit():
+    # Hand-worked: 256 slots in 64-token blocks, 150 real tokens, units of 64 tokens, radius 0,
+    # no anchors.  Blocks 0, 1 and 2 hold units 0, 1 and 2 (block 2: tokens 128..149).  Block 3
+    # holds only padding and takes the unit of the last real token, 149 // 64 = 2.  With
+    # radius 0 a block attends the blocks of its own unit: {0}, {1}, {2, 3}, {2, 3}.
+    m = window_anchor_mask(256, 150, 64, 64, 0, 0, 0)
+    assert m.astype(int).tolist() == [[1, 0, 0, 0], [0, 1, 0, 0], [0, 0, 1, 1], [0, 0, 1, 1]]
+
+
+@pytest.mark.parametrize("n_pad,n_valid,bs,U,r,G,s", [
+    (1024, 700, 64, 100, 0, 3, 123),      # five trailing padding-only blocks
+    (8192, 5000, 128, 1560, 2, 1, 0),     # frame windows, 25 padding-only blocks
+    (640, 64, 64, 64, 1, 10, 7),          # one real block, every other block padding only
+])
+def test_window_rows_with_padding_only_blocks(n_pad, n_valid, bs, U, r, G, s):
+    m = window_anchor_mask(n_pad, n_valid, bs, U, r, G, s)
+    total, lengths = _window_count_closed_form(n_pad, n_valid, bs, U, r, G, s)
+    assert m.sum(axis=1).tolist() == lengths and int(m.sum()) == total
+
+
 def _band_count(nb, r, anchors):
     band = nb * (2 * r + 1) - r * (r + 1)
     extra = sum(nb - (min(nb - 1, a + r) - max(0, a - r) + 1) for a in anchors)
