@@ -55,12 +55,20 @@ MUTANTS = {
     "attn: K in place of V": (ATT, "out[b, h, rows] = (e @ v[b, h, keys])", "out[b, h, rows] = (e @ k[b, h, keys])"),
     "attn: max added instead of subtracted": (ATT, "e = np.exp(s - m)", "e = np.exp(s + m)"),
     "attn: empty row LSE 0": (ATT, "lse[b, h, rows] = -np.inf", "lse[b, h, rows] = 0.0"),
+    "broadcast: LSE not copied": (ATT, "                    lse[b, h, i * block_size:(i + 1) * block_size] = lse[b, h, j * block_size:(j + 1) * block_size]\n",
+                                  ""),
+    "broadcast: rows copied from the block after the source": (
+        ATT, "= out[b, h, j * block_size:(j + 1) * block_size]", "= out[b, h, (j + 1) % nb * block_size:((j + 1) % nb + 1) * block_size]"),
+    "squad: global pass values are V": (ATT, "@ o_local[b, h, idx]", "@ v[b, h, idx]"),
+    "squad: global pass over windows, not positions": (ATT, "idx = np.arange(p, n, window)",
+                                                       "idx = np.arange(p * m, (p + 1) * m)"),
     # token reorder
     "reorder: w tiles before h tiles": (REO, "for h0 in range(0, H, th):\n            for w0 in range(0, W, tw):",
                                         "for w0 in range(0, W, tw):\n            for h0 in range(0, H, th):"),
     "reorder: last tile row dropped": (REO, "min(h0 + th, H)", "min(h0 + th, H - 1)"),
     "reorder: raster index transposed": (REO, "perm.append(t * H * W + h * W + w)", "perm.append(t * H * W + w * H + h)"),
     "reorder: padding rows not zeroed": (REO, "dst = np.zeros((src.shape[0], n_pad)", "dst = np.ones((src.shape[0], n_pad)"),
+    "reorder: inverse gathers instead of scattering": (REO, "dst[:, perm[k]] = src[:, k]", "dst[:, k] = src[:, perm[k]]"),
     # masks and CSR
     "mask: window bounds strict": (MSK, "lo[j] <= hi[i] + radius and hi[j] >= lo[i] - radius",
                                    "lo[j] < hi[i] + radius and hi[j] > lo[i] - radius"),
@@ -73,12 +81,18 @@ MUTANTS = {
                                        "js = [j for j in range(nb) if masks[h, j, i]]"),
     "mask: LVSA window grows left first": (MSK, "if (turn_right and can_right) or not can_left:",
                                            "if (not turn_right and can_right) or not can_left:"),
+    "mask: LVSA global frames rotate backwards": (MSK, "anchors = {(a * T // num_anchors + step) % T",
+                                                  "anchors = {(a * T // num_anchors - step) % T"),
+    "mask: two-stage groups shifted": (MSK, "if j // group == i // group:", "if (j + 1) // group == i // group:"),
     # calibration
     "calib: energies not normalised": (CAL, "a = e / e.sum(axis=1, keepdims=True)", "a = e"),
     "calib: padding keys in the softmax": (CAL, "keys = k[b, h, :n_valid]", "keys = k[b, h, :]"),
     "calib: ascending energy order": (CAL, "key=lambda j: (-e[j], j)", "key=lambda j: (e[j], j)"),
     "calib: ties by descending index": (CAL, "key=lambda j: (-e[j], j)", "key=lambda j: (-e[j], -j)"),
     "calib: threshold strict": (CAL, "if prefix[kk] >= target:", "if prefix[kk] > target:"),
+    "calib: padding query rows counted": (CAL, "r0, r1 = i * bs, min((i + 1) * bs, n_valid)", "r0, r1 = i * bs, (i + 1) * bs"),
+    "calib: absolute threshold": (CAL, "target = float(eps) * prefix[n]", "target = float(eps)"),
+    "calib: block mean instead of sum": (CAL, "energy[b, h, i, j] = a[:, c0:c1].sum()", "energy[b, h, i, j] = a[:, c0:c1].mean()"),
     "calib: agreement strict": (CAL, "return count >= float(rho) * float(p)", "return count > float(rho) * float(p)"),
 }
 
