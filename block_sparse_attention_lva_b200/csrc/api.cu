@@ -90,8 +90,10 @@ lva_status lva_reorder_tokens(const void* src, void* dst, int64_t planes, int T,
   if (n_pad < n || n_pad >= (int64_t(1) << 31)) return fail(LVA_ERR_INVALID_ARG, "reorder: need T*H*W <= n_pad < 2^31");
   const int64_t row_bytes = row_elems * elem_bytes;
   if (row_bytes > (int64_t(1) << 20)) return fail(LVA_ERR_UNSUPPORTED, "reorder: rows above 1 MiB");
-  if ((n_pad * row_bytes) / elem_bytes / 2 >= (int64_t(1) << 31) * 256)
-    return fail(LVA_ERR_UNSUPPORTED, "reorder: plane too large");
+  // One thread per (row, chunk); chunks are at least elem_bytes wide, and the launch's
+  // blocks of 256 threads must fit gridDim.x.
+  if ((n_pad * row_elems + 255) / 256 > int64_t(0x7fffffff))
+    return fail(LVA_ERR_UNSUPPORTED, "reorder: n_pad * row_elems too large for one launch");
   if (planes == 0) return ok();
   if (src == nullptr || dst == nullptr) return fail(LVA_ERR_INVALID_ARG, "reorder: null pointer");
   if (!aligned(src, elem_bytes) || !aligned(dst, elem_bytes))

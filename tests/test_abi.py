@@ -83,6 +83,12 @@ def test_reorder_argument_checks_fail_before_launch():
     assert f(vp, vp, 2, 4, 8, 8, 0, 4, 4, 256, 64, 2, 0, None) == 1     # zero tile
     assert f(None, vp, 2, 4, 8, 8, 1, 4, 4, 256, 64, 2, 0, None) == 1   # null
     assert f(vp, vp, 0, 4, 8, 8, 1, 4, 4, 256, 64, 2, 0, None) == 0     # no planes: no-op
+    # grid limit: one thread per (row, element chunk), 256-thread blocks, gridDim.x < 2^31
+    # (planes = 0 returns after the size checks, before any pointer is used)
+    assert f(vp, vp, 0, 1, 1, 1, 1, 1, 1, 1 << 30, 511, 2, 0, None) == 0
+    assert f(vp, vp, 0, 1, 1, 1, 1, 1, 1, 1 << 30, 512, 2, 0, None) == 2
+    assert b"too large" in lib.lva_last_error_message()
+    assert f(vp, vp, 0, 1, 1, 1, 1, 1, 1, 1 << 30, 512, 4, 0, None) == 2
 
 
 def test_mask_capacity_check():
