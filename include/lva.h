@@ -75,7 +75,9 @@ int lva_version(void);
  * src, dst: device, must not overlap, aligned to elem_bytes.  n_pad >= N.
  * planes * n_pad * row_elems * elem_bytes must fit in int64.
  * Errors: LVA_ERR_INVALID_ARG for null pointers, non-positive sizes, n_pad < N, bad
- * elem_bytes or misalignment.  planes == 0 is a no-op.
+ * elem_bytes or misalignment.  LVA_ERR_UNSUPPORTED when N or n_pad reaches 2^31, a row
+ * exceeds 1 MiB, or n_pad * row_elems exceeds (2^31 - 1) * 256, the most one launch
+ * covers.  planes == 0 is a no-op once the sizes have been checked.
  */
 lva_status lva_reorder_tokens(const void* src, void* dst, int64_t planes,
                               int T, int H, int W, int tile_t, int tile_h, int tile_w,
