@@ -144,8 +144,10 @@ int64_t lva_block_mask_max_nnz(const lva_mask_params* params);
  * *nnz_out = row_ptr[mask_heads*nb].  Columns of a row are ascending and unique.
  * dense_mask (device) is read only for STATIC ([mask_heads, nb, nb] uint8) and may be NULL
  * otherwise.
- * Errors: LVA_ERR_INVALID_ARG for bad parameters or pointers; LVA_ERR_CAPACITY when
- * col_capacity < lva_block_mask_max_nnz(params) (nothing is launched).
+ * Errors: LVA_ERR_INVALID_ARG for bad parameters or pointers; LVA_ERR_UNSUPPORTED for a
+ * block_size other than 64 or 128, or mask_heads*nb*nb >= 2^31 (the CSR's int32 entries);
+ * LVA_ERR_CAPACITY when col_capacity < lva_block_mask_max_nnz(params).  Nothing is
+ * launched in any of these cases.
  */
 lva_status lva_build_block_mask(const lva_mask_params* params, const uint8_t* dense_mask,
                                 int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
