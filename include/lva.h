@@ -37,7 +37,7 @@ extern "C" {
 typedef enum {
   LVA_OK = 0,
   LVA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, inconsistent sizes, bad CSR */
-  LVA_ERR_UNSUPPORTED = 2,   /* a size or mode this build has no kernel for */
+  LVA_ERR_UNSUPPORTED = 2,   /* a size or mode the library has no kernel for */
   LVA_ERR_CAPACITY = 3,      /* an output buffer is too small */
   LVA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
   LVA_ERR_TIMEOUT = 5        /* a kernel wait ran past its limit (device error word) */
