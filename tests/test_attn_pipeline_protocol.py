@@ -1,0 +1,363 @@
+"""Executable model of the attention kernel's mbarrier protocol (no GPU).
+
+``bsa_fwd_kernel`` (csrc/attn.cu) runs five kinds of roles that hand buffers to each other
+through mbarriers whose waits test a phase *parity*:
+
+* the Q/K producer (warp 0): Q once per item, then K tiles into a 3-slot ring;
+* the V producer (warp 10): V tiles into a 3-slot ring;
+* the Q K^T issuer (warp 1): S_b = Q K^T into TMEM buffer b = T mod 2;
+* the P V issuer (warp 11): O += P_b V, with P_b read from TMEM;
+* the softmax warps (2..9), each owning rows of S, P and O: read S_b, write P_b, rescale
+  O rarely, read O in the epilogue.
+
+Positions T count key blocks over all the items a CTA walks, so ring slots (T mod 3), S/P
+buffers (T mod 2) and barrier phases continue from one item to the next; ``q_empty`` and
+``o_free`` hand the single Q tile and the O accumulator from one item to the next.  Items
+with no key blocks (empty rows, corrupt rows, blocks skipped for repetitive heads) take
+no part in the pipeline.
+
+The model replays each role's waits, arrivals and buffer accesses in the kernel's order.
+TMA loads land in any order; each issuer's MMAs complete in issue order, and a
+``tcgen05.commit`` arrives once every MMA its thread issued before it has completed.  A
+seeded random scheduler runs many item runs (empty items, rows of 1 to 5 key blocks, runs
+of 1, 4 and 8 items, random rescale decisions per warp) under many interleavings and checks:
+
+* progress: every run ends, with nothing in flight (no deadlock);
+* no phase aliasing: a wait for phase k starts only when its barrier has completed k or
+  k + 1 phases and ends at exactly k + 1 (a parity test cannot tell k from k + 2);
+* no buffer hazard: a K/V ring slot, Q, or a warp's rows of S_b, P_b or O are written only
+  when no read of them is in flight (writes by one MMA issuer may overlap: its MMAs run in
+  order), and read only once written, with the content the reader expects.
+"""
+import random
+
+import pytest
+
+KST = VST = 3        # K and V ring slots
+WARPS = 3            # softmax warps modelled (8 in the kernel; the protocol is per warp)
+BLOCKED = "blocked"
+
+
+class Hazard(AssertionError):
+    pass
+
+
+class Barrier:
+    """An mbarrier: completed phases and the arrivals of the current phase."""
+
+    def __init__(self, name, count):
+        self.name, self.count, self.arrived, self.completed = name, count, 0, 0
+
+    def arrive(self):
+        self.arrived += 1
+        if self.arrived == self.count:
+            self.arrived, self.completed = 0, self.completed + 1
+
+
+class Buffer:
+    """What a buffer holds, the reads of it in flight, and the writes to it in flight."""
+
+    def __init__(self, name):
+        self.name, self.version, self.reads, self.writes, self.writer = name, None, 0, 0, None
+
+    def begin_write(self, version, writer, expect=None):
+        if self.reads:
+            raise Hazard(f"{self.name}: written ({version}) while {self.reads} read(s) of {self.version} in flight")
+        if self.writes and self.writer != writer:
+            raise Hazard(f"{self.name}: written by {writer} while a write by {self.writer} is in flight")
+        if expect is not None and self.version != expect:
+            raise Hazard(f"{self.name}: read-modify-write expects {expect}, holds {self.version}")
+        self.version, self.writes, self.writer = version, self.writes + 1, writer
+
+    def end_write(self):
+        self.writes -= 1
+
+    def begin_read(self, version):
+        if self.writes:
+            raise Hazard(f"{self.name}: read while a write ({self.version}) is in flight")
+        if self.version != version:
+            raise Hazard(f"{self.name}: read expects {version}, holds {self.version}")
+        self.reads += 1
+
+    def end_read(self):
+        self.reads -= 1
+
+
+class Model:
+    def __init__(self, items, rescale, rng, omit=()):
+        self.items, self.rescale, self.rng = items, rescale, rng
+        self.omit = set(omit)        # waits taken out, to show the checks catch their absence
+        self.bar = {}
+        for name, count in [("q", 1), ("q_empty", 1), ("o_free", WARPS), ("final", 1), ("final_pv", 1)]:
+            self.bar[name] = Barrier(name, count)
+        for s in range(KST):
+            self.bar[f"k_full{s}"], self.bar[f"k_empty{s}"] = Barrier(f"k_full{s}", 1), Barrier(f"k_empty{s}", 1)
+        for s in range(VST):
+            self.bar[f"v_full{s}"], self.bar[f"v_empty{s}"] = Barrier(f"v_full{s}", 1), Barrier(f"v_empty{s}", 1)
+        for b in range(2):
+            for name, count in [("s_full", 1), ("s_free", WARPS), ("p_full", WARPS), ("o_done", 1)]:
+                self.bar[f"{name}{b}"] = Barrier(f"{name}{b}", count)
+        names = ["Q"] + [f"K{s}" for s in range(KST)] + [f"V{s}" for s in range(VST)]
+        names += [f"{x}{b}w{w}" for x in "SP" for b in range(2) for w in range(WARPS)]
+        names += [f"Ow{w}" for w in range(WARPS)]
+        self.buf = {n: Buffer(n) for n in names}
+        self.loads = []                       # TMA copies in flight: (buffer, barrier)
+        self.mma = {"qk": [], "pv": []}       # per issuer, in issue order: completion callbacks
+
+    # -- barrier waits ------------------------------------------------------------------------
+    def wait(self, name, phase, tag):
+        if tag in self.omit:
+            return
+        bar = self.bar[name]
+        if not (phase <= bar.completed <= phase + 1):
+            raise Hazard(f"{name}: wait for phase {phase} begins with {bar.completed} completed")
+        while bar.completed == phase:
+            yield BLOCKED
+        if bar.completed != phase + 1:
+            raise Hazard(f"{name}: wait for phase {phase} ends with {bar.completed} completed")
+
+    # -- asynchronous units -------------------------------------------------------------------
+    def tma(self, buf, version, barrier):
+        self.buf[buf].begin_write(version, "tma")
+        self.loads.append((buf, barrier))
+
+    def issue_mma(self, issuer, reads, writes):
+        """reads: [(buffer, version)]; writes: [(buffer, new version, expected or None)]."""
+        for name, version in reads:
+            self.buf[name].begin_read(version)
+        for name, version, expect in writes:
+            self.buf[name].begin_write(version, issuer, expect)
+
+        def complete():
+            for name, _ in reads:
+                self.buf[name].end_read()
+            for name, _, _ in writes:
+                self.buf[name].end_write()
+        self.mma[issuer].append([complete])
+
+    def commit(self, issuer, barrier):
+        if self.mma[issuer]:
+            self.mma[issuer][-1].append(lambda: self.bar[barrier].arrive())
+        else:
+            self.bar[barrier].arrive()
+
+    def events(self):
+        return [("load", i) for i in range(len(self.loads))] + [("mma", k) for k in ("qk", "pv") if self.mma[k]]
+
+    def fire(self, ev):
+        kind, x = ev
+        if kind == "load":
+            buf, barrier = self.loads.pop(x)
+            self.buf[buf].end_write()
+            self.bar[barrier].arrive()
+        else:
+            for f in self.mma[x].pop(0):
+                f()
+
+    # -- the roles ----------------------------------------------------------------------------
+    def qk_producer(self):
+        T = nq = 0
+        for it, n in enumerate(self.items):
+            if n == 0:
+                continue
+            if nq > 0:
+                yield from self.wait("q_empty", nq - 1, "q_empty")       # the previous item's Q K^T is done
+            self.tma("Q", ("q", it), "q")
+            nq += 1
+            for _ in range(n):
+                s = T % KST
+                if T >= KST:
+                    yield from self.wait(f"k_empty{s}", T // KST - 1, "k_empty")
+                self.tma(f"K{s}", ("k", T), f"k_full{s}")
+                T += 1
+                yield
+
+    def v_producer(self):
+        T = 0
+        for n in self.items:
+            for _ in range(n):
+                s = T % VST
+                if T >= VST:
+                    yield from self.wait(f"v_empty{s}", T // VST - 1, "v_empty")
+                self.tma(f"V{s}", ("v", T), f"v_full{s}")
+                T += 1
+                yield
+
+    def qk_issuer(self):
+        T = nq = 0
+        for it, n in enumerate(self.items):
+            if n == 0:
+                continue
+            yield from self.wait("q", nq, "q_full")
+            for _ in range(n):
+                s, b = T % KST, T & 1
+                yield from self.wait(f"k_full{s}", T // KST, "k_full")
+                if T >= 2:
+                    yield from self.wait(f"s_free{b}", (T >> 1) - 1, "s_free")
+                self.issue_mma("qk", [("Q", ("q", it)), (f"K{s}", ("k", T))],
+                               [(f"S{b}w{w}", ("s", T), None) for w in range(WARPS)])
+                self.commit("qk", f"s_full{b}")
+                self.commit("qk", f"k_empty{s}")
+                T += 1
+                yield
+            self.commit("qk", "q_empty")
+            nq += 1
+        self.commit("qk", "final")
+        yield from self.wait("final", 0, "final")                     # drain before TMEM is released
+
+    def pv_issuer(self):
+        T = nq = 0
+        for n in self.items:
+            if n == 0:
+                continue
+            if nq > 0:
+                yield from self.wait("o_free", nq - 1, "o_free")       # the previous item's O was read
+            for t in range(n):
+                s, b = T % VST, T & 1
+                yield from self.wait(f"p_full{b}", T >> 1, "p_full")
+                yield from self.wait(f"v_full{s}", T // VST, "v_full")
+                o_writes = [(f"Ow{w}", ("o", T), ("o", T - 1) if t > 0 else None) for w in range(WARPS)]
+                self.issue_mma("pv", [(f"P{b}w{w}", ("p", T)) for w in range(WARPS)] + [(f"V{s}", ("v", T))],
+                               o_writes)
+                self.commit("pv", f"v_empty{s}")
+                self.commit("pv", f"o_done{b}")
+                T += 1
+                yield
+            nq += 1
+        self.commit("pv", "final_pv")
+        yield from self.wait("final_pv", 0, "final_pv")
+
+    def softmax(self, w):
+        T = 0
+        for it, n in enumerate(self.items):
+            for t in range(n):
+                b = T & 1
+                yield from self.wait(f"s_full{b}", T >> 1, "s_full")
+                self.buf[f"S{b}w{w}"].begin_read(("s", T))
+                yield                                        # tcgen05.ld of the S rows
+                self.buf[f"S{b}w{w}"].end_read()
+                self.bar[f"s_free{b}"].arrive()
+                if T >= 2:
+                    yield from self.wait(f"o_done{b}", (T >> 1) - 1, "p_reuse")   # P V(T-2) has read P_b
+                self.buf[f"P{b}w{w}"].begin_write(("p", T), f"sm{w}")
+                yield                                        # exponentials, tcgen05.st of P
+                self.buf[f"P{b}w{w}"].end_write()
+                if t >= 1 and self.rescale(w, it, t):
+                    yield from self.wait(f"o_done{b ^ 1}", (T - 1) >> 1, "rescale")   # P V(T-1) is done
+                    self.buf[f"Ow{w}"].begin_write(("o", T - 1), f"sm{w}", ("o", T - 1))
+                    yield                                    # O rows scaled in TMEM
+                    self.buf[f"Ow{w}"].end_write()
+                self.bar[f"p_full{b}"].arrive()
+                T += 1
+                yield
+            if n > 0:
+                yield from self.wait(f"o_done{(T - 1) & 1}", (T - 1) >> 1, "epilogue")
+                self.buf[f"Ow{w}"].begin_read(("o", T - 1))
+                yield                                        # tcgen05.ld of the O rows
+                self.buf[f"Ow{w}"].end_read()
+                self.bar["o_free"].arrive()
+            yield                                            # normalise, store O and LSE
+
+    # -- scheduler ----------------------------------------------------------------------------
+    def run(self, max_steps=500000):
+        live = [self.qk_producer(), self.v_producer(), self.qk_issuer(), self.pv_issuer()]
+        live += [self.softmax(w) for w in range(WARPS)]
+        blocked = set()
+        for _ in range(max_steps):
+            evs = self.events()
+            if not live and not evs:
+                break
+            choices = [("role", r) for r in live] + [("ev", e) for e in evs]
+            kind, x = self.rng.choice(choices)
+            if kind == "ev":
+                self.fire(x)
+                blocked.clear()
+                continue
+            try:
+                out = next(x)
+            except StopIteration:
+                live.remove(x)
+                blocked.clear()
+                if not live and evs:
+                    # every role has finished: the CTA synchronises and frees TMEM
+                    raise Hazard(f"teardown with {len(self.loads)} load(s) and "
+                                 f"{sum(map(len, self.mma.values()))} MMA(s) in flight")
+                continue
+            if out == BLOCKED:
+                blocked.add(id(x))
+                if not evs and all(id(r) in blocked for r in live):
+                    raise Hazard("deadlock: every role waits and nothing is in flight")
+            else:
+                blocked.clear()
+        else:
+            raise Hazard("no termination")
+        for name, b in self.buf.items():
+            if b.reads or b.writes:
+                raise Hazard(f"{name}: access in flight at exit")
+
+
+def _run(items, seed, omit=()):
+    rng = random.Random(seed)
+    decisions = {}
+
+    def rescale(w, it, t):
+        return decisions.setdefault((w, it, t), rng.random() < 0.3)
+    Model(items, rescale, rng, omit).run()
+
+
+@pytest.mark.parametrize("kpc", [1, 4, 8])
+def test_random_item_runs_and_schedules(kpc):
+    rng = random.Random(1000 + kpc)
+    for case in range(40):
+        items = [rng.choice([0, 0, 1, 1, 2, 3, 5]) for _ in range(kpc)]
+        for sched in range(6):
+            _run(items, seed=case * 100 + sched)
+
+
+@pytest.mark.parametrize("items", [
+    [1], [2], [5], [0], [0, 0, 0, 0],
+    [1, 1, 1, 1, 1, 1, 1, 1],           # one key block per item: Q and O hand-offs at every block
+    [0, 3, 0, 1, 0, 0, 2, 0],           # empty items between short rows
+    [5, 0, 0, 0, 0, 0, 0, 1],
+    [2, 2, 2, 2], [3, 1, 3, 1],         # positions cross ring and buffer boundaries inside items
+])
+def test_edge_item_runs(items):
+    for sched in range(30):
+        _run(items, seed=sched)
+
+
+# Each of these waits is needed on the normal path: without it (in the model only) some
+# schedule breaks a check.
+WAITS = ["q_empty", "k_empty", "v_empty", "q_full", "k_full", "s_free", "p_full", "v_full",
+         "s_full", "p_reuse", "rescale", "epilogue"]
+
+
+@pytest.mark.parametrize("omit", WAITS)
+def test_every_wait_is_needed(omit):
+    caught = 0
+    for sched in range(400):
+        try:
+            _run([5, 1, 3, 2], seed=sched, omit=(omit,))
+        except Hazard:
+            caught += 1
+            if caught >= 3:
+                break
+    assert caught > 0, f"no schedule needs the {omit} wait"
+
+
+@pytest.mark.parametrize("omit", ["o_free", "final", "final_pv"])
+def test_waits_implied_on_the_normal_path(omit):
+    """Three waits are implied by others when no wait times out:
+
+    * o_free (an item's O read before the next item overwrites it) by p_full: a softmax
+      warp arrives on p_full for the next item's first block only after its own epilogue
+      has read O;
+    * the issuers' final drains by the softmax: it waits for every S (s_full) and, in each
+      epilogue, for the item's last P V (o_done), so every MMA has completed before the
+      softmax warps finish and the CTA frees TMEM.
+
+    The kernel keeps all three: o_free as an explicit hand-off, and the drains for the abort
+    path, where the softmax warps may stop early.  Without them no schedule breaks a check."""
+    for sched in range(200):
+        _run([5, 1, 3, 2], seed=sched, omit=(omit,))
+        _run([1, 1, 1, 1, 1, 1, 1, 1], seed=sched, omit=(omit,))
