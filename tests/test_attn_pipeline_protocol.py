@@ -33,126 +33,40 @@ import random
 
 import pytest
 
+from tests.protocol_model import Hazard, ProtocolModel, random_decisions
+
 KST = VST = 3        # K and V ring slots
 WARPS = 3            # softmax warps modelled (8 in the kernel; the protocol is per warp)
-BLOCKED = "blocked"
 
 
-class Hazard(AssertionError):
-    pass
+class Model(ProtocolModel):
+    issuers = ("qk", "pv")
 
-
-class Barrier:
-    """An mbarrier: completed phases and the arrivals of the current phase."""
-
-    def __init__(self, name, count):
-        self.name, self.count, self.arrived, self.completed = name, count, 0, 0
-
-    def arrive(self):
-        self.arrived += 1
-        if self.arrived == self.count:
-            self.arrived, self.completed = 0, self.completed + 1
-
-
-class Buffer:
-    """What a buffer holds, the reads of it in flight, and the writes to it in flight."""
-
-    def __init__(self, name):
-        self.name, self.version, self.reads, self.writes, self.writer = name, None, 0, 0, None
-
-    def begin_write(self, version, writer, expect=None):
-        if self.reads:
-            raise Hazard(f"{self.name}: written ({version}) while {self.reads} read(s) of {self.version} in flight")
-        if self.writes and self.writer != writer:
-            raise Hazard(f"{self.name}: written by {writer} while a write by {self.writer} is in flight")
-        if expect is not None and self.version != expect:
-            raise Hazard(f"{self.name}: read-modify-write expects {expect}, holds {self.version}")
-        self.version, self.writes, self.writer = version, self.writes + 1, writer
-
-    def end_write(self):
-        self.writes -= 1
-
-    def begin_read(self, version):
-        if self.writes:
-            raise Hazard(f"{self.name}: read while a write ({self.version}) is in flight")
-        if self.version != version:
-            raise Hazard(f"{self.name}: read expects {version}, holds {self.version}")
-        self.reads += 1
-
-    def end_read(self):
-        self.reads -= 1
-
-
-class Model:
     def __init__(self, items, rescale, rng, omit=()):
-        self.items, self.rescale, self.rng = items, rescale, rng
-        self.omit = set(omit)        # waits taken out, to show the checks catch their absence
-        self.bar = {}
+        super().__init__(rng, omit)
+        self.items, self.rescale = items, rescale
         for name, count in [("q", 1), ("q_empty", 1), ("o_free", WARPS), ("final", 1), ("final_pv", 1)]:
-            self.bar[name] = Barrier(name, count)
+            self.barrier(name, count)
         for s in range(KST):
-            self.bar[f"k_full{s}"], self.bar[f"k_empty{s}"] = Barrier(f"k_full{s}", 1), Barrier(f"k_empty{s}", 1)
+            self.barrier(f"k_full{s}", 1)
+            self.barrier(f"k_empty{s}", 1)
         for s in range(VST):
-            self.bar[f"v_full{s}"], self.bar[f"v_empty{s}"] = Barrier(f"v_full{s}", 1), Barrier(f"v_empty{s}", 1)
+            self.barrier(f"v_full{s}", 1)
+            self.barrier(f"v_empty{s}", 1)
         for b in range(2):
             for name, count in [("s_full", 1), ("s_free", WARPS), ("p_full", WARPS), ("o_done", 1)]:
-                self.bar[f"{name}{b}"] = Barrier(f"{name}{b}", count)
-        names = ["Q"] + [f"K{s}" for s in range(KST)] + [f"V{s}" for s in range(VST)]
-        names += [f"{x}{b}w{w}" for x in "SP" for b in range(2) for w in range(WARPS)]
-        names += [f"Ow{w}" for w in range(WARPS)]
-        self.buf = {n: Buffer(n) for n in names}
-        self.loads = []                       # TMA copies in flight: (buffer, barrier)
-        self.mma = {"qk": [], "pv": []}       # per issuer, in issue order: completion callbacks
+                self.barrier(f"{name}{b}", count)
+        for name in ["Q"] + [f"K{s}" for s in range(KST)] + [f"V{s}" for s in range(VST)]:
+            self.buffer(name)
+        for w in range(WARPS):
+            for b in range(2):
+                self.buffer(f"S{b}w{w}")
+                self.buffer(f"P{b}w{w}")
+            self.buffer(f"Ow{w}")
 
-    # -- barrier waits ------------------------------------------------------------------------
-    def wait(self, name, phase, tag):
-        if tag in self.omit:
-            return
-        bar = self.bar[name]
-        if not (phase <= bar.completed <= phase + 1):
-            raise Hazard(f"{name}: wait for phase {phase} begins with {bar.completed} completed")
-        while bar.completed == phase:
-            yield BLOCKED
-        if bar.completed != phase + 1:
-            raise Hazard(f"{name}: wait for phase {phase} ends with {bar.completed} completed")
-
-    # -- asynchronous units -------------------------------------------------------------------
-    def tma(self, buf, version, barrier):
-        self.buf[buf].begin_write(version, "tma")
-        self.loads.append((buf, barrier))
-
-    def issue_mma(self, issuer, reads, writes):
-        """reads: [(buffer, version)]; writes: [(buffer, new version, expected or None)]."""
-        for name, version in reads:
-            self.buf[name].begin_read(version)
-        for name, version, expect in writes:
-            self.buf[name].begin_write(version, issuer, expect)
-
-        def complete():
-            for name, _ in reads:
-                self.buf[name].end_read()
-            for name, _, _ in writes:
-                self.buf[name].end_write()
-        self.mma[issuer].append([complete])
-
-    def commit(self, issuer, barrier):
-        if self.mma[issuer]:
-            self.mma[issuer][-1].append(lambda: self.bar[barrier].arrive())
-        else:
-            self.bar[barrier].arrive()
-
-    def events(self):
-        return [("load", i) for i in range(len(self.loads))] + [("mma", k) for k in ("qk", "pv") if self.mma[k]]
-
-    def fire(self, ev):
-        kind, x = ev
-        if kind == "load":
-            buf, barrier = self.loads.pop(x)
-            self.buf[buf].end_write()
-            self.bar[barrier].arrive()
-        else:
-            for f in self.mma[x].pop(0):
-                f()
+    def roles(self):
+        return [self.qk_producer(), self.v_producer(), self.qk_issuer(), self.pv_issuer()] + \
+               [self.softmax(w) for w in range(WARPS)]
 
     # -- the roles ----------------------------------------------------------------------------
     def qk_producer(self):
@@ -258,51 +172,10 @@ class Model:
                 self.bar["o_free"].arrive()
             yield                                            # normalise, store O and LSE
 
-    # -- scheduler ----------------------------------------------------------------------------
-    def run(self, max_steps=500000):
-        live = [self.qk_producer(), self.v_producer(), self.qk_issuer(), self.pv_issuer()]
-        live += [self.softmax(w) for w in range(WARPS)]
-        blocked = set()
-        for _ in range(max_steps):
-            evs = self.events()
-            if not live and not evs:
-                break
-            choices = [("role", r) for r in live] + [("ev", e) for e in evs]
-            kind, x = self.rng.choice(choices)
-            if kind == "ev":
-                self.fire(x)
-                blocked.clear()
-                continue
-            try:
-                out = next(x)
-            except StopIteration:
-                live.remove(x)
-                blocked.clear()
-                if not live and evs:
-                    # every role has finished: the CTA synchronises and frees TMEM
-                    raise Hazard(f"teardown with {len(self.loads)} load(s) and "
-                                 f"{sum(map(len, self.mma.values()))} MMA(s) in flight")
-                continue
-            if out == BLOCKED:
-                blocked.add(id(x))
-                if not evs and all(id(r) in blocked for r in live):
-                    raise Hazard("deadlock: every role waits and nothing is in flight")
-            else:
-                blocked.clear()
-        else:
-            raise Hazard("no termination")
-        for name, b in self.buf.items():
-            if b.reads or b.writes:
-                raise Hazard(f"{name}: access in flight at exit")
-
 
 def _run(items, seed, omit=()):
     rng = random.Random(seed)
-    decisions = {}
-
-    def rescale(w, it, t):
-        return decisions.setdefault((w, it, t), rng.random() < 0.3)
-    Model(items, rescale, rng, omit).run()
+    Model(items, random_decisions(rng, 0.3), rng, omit).run()
 
 
 @pytest.mark.parametrize("kpc", [1, 4, 8])
