@@ -212,3 +212,25 @@ def test_lvsa_block_mask_from_frames():
     for i in range(T * fb):
         for j in range(T * fb):
             assert m[i, j] == ((j // fb) in sets[i // fb])
+
+
+def _cyclic_gaps(points, n):
+    p = sorted(points)
+    return [(p[(k + 1) % len(p)] - p[k]) % n or n for k in range(len(p))]
+
+
+@pytest.mark.parametrize("n,G", [(10, 4), (21, 4), (81, 4), (591, 4), (988, 6), (7, 7), (13, 5)])
+def test_anchors_spread_evenly_and_rotate(n, G):
+    """Both anchor sets -- key blocks (window kind) and global frames (LVSA frames kind) --
+    are G distinct positions spread as evenly as the count allows (cyclic gaps differ by at
+    most one, LVSA page section 2: anchors spread over the sequence), and the step s shifts
+    every one of them by s (the rotation of the global set)."""
+    for s in (0, 1, 3, n - 1):
+        block_anchors = anchor_set(n, G, s)
+        frame_anchors, _, _ = lvsa_frame_sets(n, G, s, 1)
+        for anchors in (block_anchors, frame_anchors):
+            assert len(anchors) == G
+            gaps = _cyclic_gaps(anchors, n)
+            assert max(gaps) - min(gaps) <= 1, (n, G, s, sorted(anchors))
+            assert anchors == {(a + s) % n for a in (anchor_set(n, G, 0) if anchors is block_anchors
+                                                     else lvsa_frame_sets(n, G, 0, 1)[0])}

@@ -62,6 +62,8 @@ MUTANTS = {
     "squad: global pass values are V": (ATT, "@ o_local[b, h, idx]", "@ v[b, h, idx]"),
     "squad: global pass over windows, not positions": (ATT, "idx = np.arange(p, n, window)",
                                                        "idx = np.arange(p * m, (p + 1) * m)"),
+    "squad: local pass over positions": (ATT, "idx = np.arange(a * window, (a + 1) * window)",
+                                         "idx = np.arange(a, n, m)"),
     # token reorder
     "reorder: w tiles before h tiles": (REO, "for h0 in range(0, H, th):\n            for w0 in range(0, W, tw):",
                                         "for w0 in range(0, W, tw):\n            for h0 in range(0, H, th):"),
@@ -69,6 +71,7 @@ MUTANTS = {
     "reorder: raster index transposed": (REO, "perm.append(t * H * W + h * W + w)", "perm.append(t * H * W + w * H + h)"),
     "reorder: padding rows not zeroed": (REO, "dst = np.zeros((src.shape[0], n_pad)", "dst = np.ones((src.shape[0], n_pad)"),
     "reorder: inverse gathers instead of scattering": (REO, "dst[:, perm[k]] = src[:, k]", "dst[:, k] = src[:, perm[k]]"),
+    "reorder: tile depth ignored": (REO, "for t in range(t0, min(t0 + tt, T)):", "for t in range(t0, min(t0 + 1, T)):"),
     # masks and CSR
     "mask: window bounds strict": (MSK, "lo[j] <= hi[i] + radius and hi[j] >= lo[i] - radius",
                                    "lo[j] < hi[i] + radius and hi[j] > lo[i] - radius"),
@@ -84,6 +87,14 @@ MUTANTS = {
     "mask: LVSA global frames rotate backwards": (MSK, "anchors = {(a * T // num_anchors + step) % T",
                                                   "anchors = {(a * T // num_anchors - step) % T"),
     "mask: two-stage groups shifted": (MSK, "if j // group == i // group:", "if (j + 1) // group == i // group:"),
+    "mask: anchors spaced by nb // G": (MSK, "anchors.add((a * nb // num_anchors + step) % nb)",
+                                        "anchors.add((a * (nb // num_anchors) + step) % nb)"),
+    "mask: two-stage stride of one block": (MSK, "m[i, (i + group) % nb] = True", "m[i, (i + 1) % nb] = True"),
+    "mask: LVSA global frames spaced by T // G": (MSK, "anchors = {(a * T // num_anchors + step) % T",
+                                                  "anchors = {(a * (T // num_anchors) + step) % T"),
+    "mask: LVSA block's last frame dropped": (MSK, "return range(first // frame_tokens, last // frame_tokens + 1)",
+                                              "return range(first // frame_tokens, last // frame_tokens)"),
+    "mask: LVSA budget one short": (MSK, "target = min(budget, T)", "target = min(budget, T) - 1"),
     # calibration
     "calib: energies not normalised": (CAL, "a = e / e.sum(axis=1, keepdims=True)", "a = e"),
     "calib: padding keys in the softmax": (CAL, "keys = k[b, h, :n_valid]", "keys = k[b, h, :]"),
@@ -93,8 +104,15 @@ MUTANTS = {
     "calib: padding query rows counted": (CAL, "r0, r1 = i * bs, min((i + 1) * bs, n_valid)", "r0, r1 = i * bs, (i + 1) * bs"),
     "calib: absolute threshold": (CAL, "target = float(eps) * prefix[n]", "target = float(eps)"),
     "calib: block mean instead of sum": (CAL, "energy[b, h, i, j] = a[:, c0:c1].sum()", "energy[b, h, i, j] = a[:, c0:c1].mean()"),
+    "calib: one block too many": (CAL, "for j in order[:kcount]:", "for j in order[:kcount + 1]:"),
     "calib: agreement strict": (CAL, "return count >= float(rho) * float(p)", "return count > float(rho) * float(p)"),
 }
+
+
+# Not listed: mistakes that change nothing, so no pin can see them.  Examples are a
+# partial last block taking the unit of its last padding token (that unit lies beyond
+# every block's range anyway), and the energy softmax without the max subtraction (the
+# normalisation cancels it).
 
 
 def _run(case):
