@@ -104,8 +104,13 @@ def _need(cond: bool, msg: str):
 
 
 def _cuda_tensor(t, name: str, dtype=None, numel: int = None):
-    """Checks that ``t`` is a contiguous CUDA tensor (of ``dtype``, with >= ``numel`` elements)."""
+    """Checks that ``t`` is a contiguous CUDA tensor on the current device (of ``dtype``, with
+    >= ``numel`` elements).  The library launches on the current device, so a tensor of
+    another device would hand its kernels a foreign address."""
+    import torch
     _need(t is not None and t.is_cuda, f"{name} must be a CUDA tensor")
+    current = torch.cuda.current_device()
+    _need(t.device.index == current, f"{name} is on cuda:{t.device.index}, the current device is cuda:{current}")
     _need(t.is_contiguous(), f"{name} must be contiguous")
     if dtype is not None:
         _need(t.dtype == dtype, f"{name} must be {dtype}, got {t.dtype}")

@@ -52,3 +52,30 @@ CALLS = {
 def test_host_tensors_are_refused(name):
     with pytest.raises(ValueError, match="must be a CUDA tensor"):
         CALLS[name]()
+
+
+class _FakeCudaTensor:
+    """Duck-typed stand-in for a CUDA tensor (only what the binding's check reads)."""
+    is_cuda = True
+
+    def __init__(self, index):
+        self.device = torch.device("cuda", index)
+        self.dtype = torch.bfloat16
+
+    def is_contiguous(self):
+        return True
+
+    def numel(self):
+        return 16
+
+
+def test_tensors_of_another_device_are_refused(monkeypatch):
+    from block_sparse_attention_lva_b200 import _binding
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    _binding._cuda_tensor(_FakeCudaTensor(0), "q", torch.bfloat16, 16)          # current device: accepted
+    with pytest.raises(ValueError, match="q is on cuda:1, the current device is cuda:0"):
+        _binding._cuda_tensor(_FakeCudaTensor(1), "q", torch.bfloat16, 16)
+    with pytest.raises(ValueError, match="q must be torch.float32, got torch.bfloat16"):
+        _binding._cuda_tensor(_FakeCudaTensor(0), "q", torch.float32)
+    with pytest.raises(ValueError, match="needs 17"):
+        _binding._cuda_tensor(_FakeCudaTensor(0), "q", None, 17)
