@@ -31,7 +31,9 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_shard_and_reduce():
     world, port = 2, _free_port()
-    with mp.Manager() as m:
+    # the manager process is spawned too: forking a process that already runs threads
+    # (torch's pools, earlier tests) can deadlock the child
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
