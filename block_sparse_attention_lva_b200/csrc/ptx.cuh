@@ -110,7 +110,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
 }
 
 // 2D tiled load of one box into shared memory; completion is signalled as transaction
-// bytes on `bar`.  No multicast.
+// bytes on `bar`.  The box lands in this CTA's shared memory only.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int32_t x, int32_t y,
                                             uint32_t bar) {
   asm volatile(
