@@ -13,7 +13,7 @@ section 2 A, the offline calibration phase:
 The result is a static per-(timestep, layer, head) block mask: the input of the static
 mask kind of the CSR builder.
 
-Readings where the page is silent (listed in the design notes):
+Readings where the page is silent (the plainest form section 2 A supports):
 
 * attention scores are the row-softmax probabilities over all real keys (c < n_valid),
   A[r][c] = exp(s_rc - LSE_r) with s_rc = scale * <q_r, k_c>;

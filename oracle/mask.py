@@ -16,7 +16,7 @@ A block mask M[h_m][i][j] says whether query block i attends key block j (blocks
   windows of size w, and a global pass linking the same relative position across windows;
   w = sqrt(n).
 
-Readings where the pages are silent (each listed in the design notes):
+Readings where the pages are silent (the plainest form the passages above support):
 
 * Windows are measured in units of ``U`` tokens (U = H*W gives latent frames when the
   tile depth is 1; U = Bs gives block windows).  Block i spans units lo(i)..hi(i) of its

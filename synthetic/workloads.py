@@ -138,45 +138,65 @@ def make_qk_calibration(w: Workload, prompt: int, heads: Optional[Iterable[int]]
     return q, k
 
 
+def _block_centroids(w: Workload) -> np.ndarray:
+    """Mean latent coordinates (t, y, x) of the real tokens of every block, [nb, 3].
+
+    Tokens are ranked in the spatiotemporal tile order of the workload (tiles of
+    ``w.tile`` in raster order of tile coordinates, tokens in raster order inside a tile)
+    by one lexicographic sort of their coordinates; this serves only to place the blocks
+    of the random mask below and is not part of any computation under test.
+    """
+    tt, th, tw = w.tile
+    t, y, x = np.meshgrid(np.arange(w.T), np.arange(w.Hg), np.arange(w.Wg), indexing="ij")
+    t, y, x = t.reshape(-1), y.reshape(-1), x.reshape(-1)
+    order = np.lexsort((x % tw, y % th, t % tt, x // tw, y // th, t // tt))
+    coords = np.stack([t[order], y[order], x[order]], axis=1).astype(np.float64)
+    cent = np.zeros((w.nb, 3))
+    for i in range(w.nb):
+        blk = coords[i * w.block_size:(i + 1) * w.block_size]
+        # a block of padding only sits at the last real token
+        cent[i] = blk.mean(axis=0) if len(blk) else coords[-1]
+    return cent
+
+
 def static_calibrated_mask(w: Workload, density: float = 0.30, seed_base: int = 1000) -> np.ndarray:
     """Random per-head static block mask [H, nb, nb] (uint8) standing in for a calibrated mask.
 
-    Blocks sit on a coarse spatiotemporal coordinate: ``u = (i + 0.5) * Bs / frame_tokens``
-    frames, split into a frame coordinate ``u`` and an in-frame coordinate ``frac(u)``.
-    Off-diagonal blocks are kept with probability ``min(1, c_h * exp(-dist / tau_h))``, where
-    ``tau_h`` varies by head and ``c_h`` is found by bisection so that the expected density,
-    counting the always-kept diagonal as 1, equals ``density``.  Draws come from numpy's
-    PCG64 seeded with ``seed_base + h``.
+    Block i sits at the centroid (t_i, y_i, x_i) of its real tokens' latent coordinates.
+    The spatiotemporal distance of blocks i, j weighs a frame like 8 latent rows or 16
+    latent columns (one tile):
+        delta_ij = sqrt((t_i - t_j)^2 + ((y_i - y_j) / 8)^2 + ((x_i - x_j) / 16)^2).
+    Block (i, j) is kept with probability p_ij = min(1, c * exp(-delta_ij / 2)), and always
+    when i == j; c is found by float64 bisection so that the expected density, counting the
+    diagonal as 1, equals ``density``.  Head h draws u_ij uniform from numpy's PCG64
+    seeded with ``seed_base + h`` and keeps the block when u_ij < p_ij.
     """
     nb = w.nb
-    u = (np.arange(nb, dtype=np.float64) + 0.5) * w.block_size / w.frame_tokens
-    frac = u - np.floor(u)
-    dt = u[:, None] - u[None, :]
-    ds = 4.0 * (frac[:, None] - frac[None, :])
-    dist = np.sqrt(dt * dt + ds * ds)
+    cent = _block_centroids(w)
+    dt = cent[:, None, 0] - cent[None, :, 0]
+    dy = (cent[:, None, 1] - cent[None, :, 1]) / 8.0
+    dx = (cent[:, None, 2] - cent[None, :, 2]) / 16.0
+    base = np.exp(-np.sqrt(dt * dt + dy * dy + dx * dx) / 2.0)
     eye = np.eye(nb, dtype=bool)
+
+    def expected(c):
+        p = np.minimum(1.0, c * base)
+        p[eye] = 1.0
+        return p.mean()
+
+    lo, hi = 0.0, 1.0
+    while expected(hi) < density:
+        hi *= 2.0
+    for _ in range(100):
+        mid = 0.5 * (lo + hi)
+        if expected(mid) < density:
+            lo = mid
+        else:
+            hi = mid
+    p = np.minimum(1.0, hi * base)
     masks = np.zeros((w.H, nb, nb), dtype=np.uint8)
     for h in range(w.H):
-        tau = 1.0 + 2.0 * h / max(1, w.H - 1)
-        base = np.exp(-dist / tau)
-
-        def expected(c):
-            p = np.minimum(1.0, c * base)
-            p[eye] = 1.0
-            return p.mean()
-
-        lo, hi = 0.0, 1.0
-        while expected(hi) < density:
-            hi *= 2.0
-        for _ in range(100):
-            mid = 0.5 * (lo + hi)
-            if expected(mid) < density:
-                lo = mid
-            else:
-                hi = mid
-        p = np.minimum(1.0, hi * base)
-        rng = np.random.default_rng(seed_base + h)
-        draw = rng.random((nb, nb))
+        draw = np.random.default_rng(seed_base + h).random((nb, nb))
         masks[h] = ((draw < p) | eye).astype(np.uint8)
     return masks
 

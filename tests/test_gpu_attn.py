@@ -3,7 +3,9 @@
 * Multi-tile shapes with ragged tails, empty rows, random pad contents, both head dims and
   both block sizes: every output element compared.
 * The five workloads at full size through the whole layer path (reorder, CSR, attention,
-  inverse reorder): sampled query blocks compared, every row checked for NaN / -inf.
+  inverse reorder): every element of O and LSE for the small workload (step 0) and the
+  static 30 % masks; sampled query blocks for every other mask, every row checked for
+  NaN / -inf.
 """
 import math
 
@@ -13,7 +15,7 @@ import torch
 
 from oracle.attention import attention_blocked
 from oracle.mask import all_mask, dense_to_csr, lvsa_frame_mask, two_stage_mask, window_anchor_mask
-from oracle.reorder import reorder_forward, tile_permutation
+from oracle.reorder import reorder_forward, reorder_inverse, tile_permutation
 from synthetic import WORKLOADS, make_qkv, mask_variants, static_calibrated_mask
 from tests.gpu_helpers import check_o_lse, require_gpu
 
@@ -165,7 +167,7 @@ def _sample_blocks(w, masks, seed, per_head=2):
     return out
 
 
-def _run_workload(name, labels, steps=(0,), per_head=2):
+def _run_workload(name, labels, steps=(0,), per_head=2, whole=False):
     import block_sparse_attention_lva_b200 as lva
     dev = require_gpu()
     w = WORKLOADS[name]
@@ -197,6 +199,12 @@ def _run_workload(name, labels, steps=(0,), per_head=2):
             assert torch.isfinite(layer.lse).all()
             lse_t = layer.lse.cpu().numpy()
             o_r = o.float().cpu().numpy()
+            if whole:
+                # every element of O (raster order) and LSE (tile order), all heads and rows
+                ro, rl = attention_blocked(tile[0], tile[1], tile[2], masks, w.block_size, w.n_valid, w.scale)
+                ro_raster = reorder_inverse(ro.reshape(P, w.n_pad, w.d), perm).reshape(o_r.shape)
+                check_o_lse(o_r, lse_t, ro_raster, rl, f"{name}/{spec['label']}/s{s} (every element)")
+                continue
             got_o, got_l, ref_o, ref_l = [], [], [], []
             for h, i in _sample_blocks(w, masks, seed=w.seed * 100 + s, per_head=per_head):
                 hm = h if masks.shape[0] > 1 else 0
@@ -214,19 +222,30 @@ def _run_workload(name, labels, steps=(0,), per_head=2):
 
 
 def test_workload_small():
-    _run_workload("small", {"frame1_anchor4"}, steps=(0, 1, 37, 49))
+    _run_workload("small", {"frame1_anchor4"}, steps=(1, 37, 49))
+
+
+def test_workload_small_every_element():
+    """The small workload at step 0: every element of O and LSE against the oracle."""
+    _run_workload("small", {"frame1_anchor4"}, steps=(0,), whole=True)
 
 
 def test_workload_static():
-    _run_workload("static", {"static30", "all"})
+    _run_workload("static", {"all"})
+
+
+def test_workload_static30_every_element():
+    """Per-head static 30 % masks: every element of O and LSE against the oracle."""
+    _run_workload("static", {"static30"}, whole=True)
 
 
 def test_workload_large():
-    _run_workload("large", {"band28_anchor4", "band171_anchor4"}, per_head=1)
+    _run_workload("large", {"band28_anchor4", "band60_anchor4", "band171_anchor4"}, per_head=1)
 
 
 def test_workload_long():
-    _run_workload("long", {"two_stage", "band23_anchor4", "all", "lvsa_c21_g4"}, per_head=1)
+    _run_workload("long", {"two_stage", "band23_anchor4", "band48_anchor4", "band130_anchor4",
+                           "band287_anchor4", "all", "lvsa_c21_g4"}, per_head=1)
 
 
 @pytest.mark.parametrize("name,grid,tile,d,bs", [
