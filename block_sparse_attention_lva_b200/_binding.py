@@ -37,6 +37,21 @@ class LvaMaskParams(ctypes.Structure):
                 ("budget_frames", ctypes.c_int)]
 
 
+class LvaLayerShape(ctypes.Structure):
+    """Mirror of ``lva_layer_shape``."""
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("block_size", ctypes.c_int),
+                ("T", ctypes.c_int), ("Hg", ctypes.c_int), ("Wg", ctypes.c_int), ("tile_t", ctypes.c_int),
+                ("tile_h", ctypes.c_int), ("tile_w", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class LvaHostStepBuffers(ctypes.Structure):
+    """Mirror of ``lva_host_step_buffers``."""
+    _fields_ = [("qkv_stage", ctypes.c_void_p), ("o_stage", ctypes.c_void_p), ("lse_stage", ctypes.c_void_p),
+                ("qkv_tile", ctypes.c_void_p), ("o_tile", ctypes.c_void_p), ("row_ptr", ctypes.c_void_p),
+                ("col_idx", ctypes.c_void_p), ("col_capacity", ctypes.c_int64), ("col_len", ctypes.c_int64),
+                ("nnz", ctypes.c_void_p), ("events", ctypes.POINTER(ctypes.c_void_p)), ("num_events", ctypes.c_int)]
+
+
 SIGNATURES = {
     "lva_status_string": (ctypes.c_char_p, [_c_int]),
     "lva_last_error_message": (ctypes.c_char_p, []),
@@ -47,6 +62,8 @@ SIGNATURES = {
     "lva_build_block_mask": (_c_int, [ctypes.POINTER(LvaMaskParams), _vp, _vp, _vp, _c_i64, _vp, _vp]),
     "lva_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
                                        _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp, _c_int, _vp]),
+    "lva_block_sparse_lse": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int, _c_int, _vp, _vp,
+                                      _c_i64, _c_int, ctypes.c_float, _vp]),
     "lva_block_sparse_attn_raster": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
                                               _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _c_int, _c_int,
                                               _c_int, _c_int, _c_int, _c_int, _vp]),
@@ -57,6 +74,9 @@ SIGNATURES = {
                                   _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp]),
     "lva_select_blocks": (_c_int, [_vp, _vp, _c_i64, _c_int, ctypes.c_double, _vp]),
     "lva_aggregate_masks": (_c_int, [_vp, _vp, _c_int, _c_i64, ctypes.c_double, _vp]),
+    "lva_layer_step_host": (_c_int, [_vp, _vp, _vp, ctypes.POINTER(LvaLayerShape), ctypes.POINTER(LvaMaskParams),
+                                     _vp, _c_int, _vp, _c_int, ctypes.POINTER(LvaHostStepBuffers), _c_int, _vp, _vp,
+                                     _vp, ctypes.POINTER(ctypes.c_void_p)]),
     "lva_device_error": (_c_int, [_vp, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
     "lva_selftest_wait": (_c_int, [_c_int, _vp]),
 }
@@ -215,6 +235,24 @@ def lva_block_sparse_attn(q, k, v, o, lse, n_valid: int, block_size: int, row_pt
     return o, lse
 
 
+def lva_block_sparse_lse(q, k, lse, n_valid: int, block_size: int, row_ptr, col_idx, mask_heads: int,
+                         scale: float):
+    """Row log-sum-exp [B, H, n_pad] (fp32) of block-sparse attention, without O (V unused)."""
+    import torch
+    B, H, n_pad, d = q.shape
+    for name, t in (("q", q), ("k", k)):
+        _cuda_tensor(t, name, torch.bfloat16)
+        _need(tuple(t.shape) == (B, H, n_pad, d), f"{name} must have shape {(B, H, n_pad, d)}")
+    _cuda_tensor(lse, "lse", torch.float32, B * H * n_pad)
+    nb = n_pad // block_size
+    _cuda_tensor(row_ptr, "row_ptr", torch.int32, mask_heads * nb + 1)
+    _cuda_tensor(col_idx, "col_idx", torch.int32)
+    _check(lib.lva_block_sparse_lse(_ptr(q), _ptr(k), _ptr(lse), B, H, n_pad, n_valid, d, block_size,
+                                    _ptr(row_ptr), _ptr(col_idx), col_idx.numel(), mask_heads,
+                                    ctypes.c_float(scale), ctypes.c_void_p(_stream(q.device))))
+    return lse
+
+
 def lva_block_sparse_attn_raster(q, k, v, o_raster, lse, n_valid: int, block_size: int, row_ptr, col_idx,
                                  mask_heads: int, scale: float, grid, tile):
     """Block-sparse attention on tile-order Q, K, V with O written in raster order
@@ -310,6 +348,39 @@ def lva_aggregate_masks(masks, out, rho: float):
     _check(lib.lva_aggregate_masks(_ptr(masks), _ptr(out), masks.shape[0], out.numel(), ctypes.c_double(rho),
                                    ctypes.c_void_p(_stream(masks.device))))
     return out
+
+
+def lva_layer_step_host(qkv_host, o_host, lse_host, shape: LvaLayerShape, params: "MaskParams", dense_mask,
+                        build_mask: bool, query_src, bufs: LvaHostStepBuffers, head_groups: int, h2d, d2h,
+                        compute=None) -> int:
+    """Enqueue one layer step from pinned host buffers (``lva_layer_step_host``); returns the
+    raw handle of the event that completes when ``o_host`` and ``lse_host`` hold the results.
+    ``h2d`` / ``d2h`` / ``compute`` are torch streams (compute: the current stream)."""
+    import torch
+    B, H, d = shape.B, shape.H, shape.d
+    N = shape.T * shape.Hg * shape.Wg
+    for name, t, shp, dt in (("qkv_host", qkv_host, (3, B, H, N, d), torch.bfloat16),
+                             ("o_host", o_host, (B, H, N, d), torch.bfloat16),
+                             ("lse_host", lse_host, (B, H, params.n_pad), torch.float32)):
+        _need(tuple(t.shape) == shp and t.dtype == dt and t.is_contiguous() and not t.is_cuda,
+              f"{name} must be a contiguous host {dt} tensor of shape {shp}")
+    if params.kind == LVA_MASK_STATIC and build_mask:
+        nb = params.n_pad // params.block_size
+        _cuda_tensor(dense_mask, "dense_mask", torch.uint8, params.mask_heads * nb * nb)
+    src_heads = 1
+    if query_src is not None:
+        _check_query_src(query_src, H, params.n_pad // params.block_size)
+        src_heads = query_src.shape[0]
+    compute = torch.cuda.current_stream() if compute is None else compute
+    cp = params.to_c()
+    done = ctypes.c_void_p(0)
+    _check(lib.lva_layer_step_host(_ptr(qkv_host), _ptr(o_host), _ptr(lse_host), ctypes.byref(shape),
+                                   ctypes.byref(cp), _ptr(dense_mask) if params.kind == LVA_MASK_STATIC else None,
+                                   int(bool(build_mask)), _ptr(query_src), src_heads, ctypes.byref(bufs),
+                                   int(head_groups), ctypes.c_void_p(compute.cuda_stream),
+                                   ctypes.c_void_p(h2d.cuda_stream), ctypes.c_void_p(d2h.cuda_stream),
+                                   ctypes.byref(done)))
+    return done.value
 
 
 def lva_device_error(stream=None):

@@ -20,7 +20,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "liblva.so")
 
 SOURCES = ["api.cu", "reorder.cu", "mask.cu", "attn.cu", "broadcast.cu", "tmap.cu", "energy.cu", "calib.cu",
-           "selftest.cu"]
+           "selftest.cu", "layer.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

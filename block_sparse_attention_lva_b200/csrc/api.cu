@@ -4,6 +4,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "kernels.h"
 #include "lva.h"
@@ -31,15 +32,37 @@ lva_status from_cuda(cudaError_t e, const char* what) {
   return fail(LVA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-// Kernel-side error word: [0] = status, [1] = detail.  One copy per device (module global);
-// its device address is looked up once per device (on every call past the cache).
-__device__ int g_device_error[2];
+// Kernel-side error word: [0] = status, [1] = detail, read and written as one 64-bit word.
+// One copy per device (module global); its device address is looked up once per device (on
+// every call past the cache).
+__device__ __align__(8) int g_device_error[2];
+
+// Where lva_device_error's exchange kernel leaves the word it took.
+__device__ unsigned long long g_device_error_taken;
+
+// Takes the error word and clears it in one atomic exchange, so a fault recorded by a
+// kernel on another stream at the same moment is either taken now or left for the next
+// read, never lost.
+__global__ void take_error_kernel(unsigned long long* word) {
+  g_device_error_taken = atomicExch(word, 0ull);
+}
+
+// lva_device_error calls are serialised: they share the taken-word slot of a device.
+std::mutex g_take_mutex;
 
 std::atomic<int*> g_err_ptr[kMaxCachedDevices] = {};
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 }  // namespace
+
+lva_status set_error_message(lva_status status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return status;
+}
 
 int* device_error_word() {
   int dev = 0;
@@ -186,7 +209,7 @@ static lva_status attn_common(const char* fn, const void* q, const void* k, cons
                               int64_t col_len, int mask_heads, float scale, const int32_t* query_src,
                               int src_heads, void* o_raster, int T, int Hg, int Wg, int tile_t,
                               int tile_h, int tile_w, int gather_windows, int gather_window,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int lse_only = 0) {
   if (B < 0 || H < 1) return fail(LVA_ERR_INVALID_ARG, "%s: need B >= 0 and H >= 1", fn);
   if (d != 64 && d != 128) return fail(LVA_ERR_UNSUPPORTED, "%s: head dim must be 64 or 128", fn);
   if (block_size != 64 && block_size != 128) return fail(LVA_ERR_UNSUPPORTED, "%s: block_size must be 64 or 128", fn);
@@ -207,9 +230,9 @@ static lva_status attn_common(const char* fn, const void* q, const void* k, cons
       return fail(LVA_ERR_INVALID_ARG, "%s: T*H*W must equal n_valid", fn);
   }
   if (B == 0) return ok();
-  if (!q || !k || !v || !(o || o_raster) || !lse || !row_ptr || (!col_idx && col_len > 0))
+  if (!q || !k || (!lse_only && (!v || !(o || o_raster))) || !lse || !row_ptr || (!col_idx && col_len > 0))
     return fail(LVA_ERR_INVALID_ARG, "%s: null pointer", fn);
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || (o && !aligned(o, 16)) ||
+  if (!aligned(q, 16) || !aligned(k, 16) || (v && !aligned(v, 16)) || (o && !aligned(o, 16)) ||
       (o_raster && !aligned(o_raster, 16)))
     return fail(LVA_ERR_INVALID_ARG, "%s: q, k, v, o must be 16-byte aligned", fn);
   if (!aligned(lse, 4) || !aligned(row_ptr, 4) || !aligned(col_idx, 4))
@@ -218,7 +241,7 @@ static lva_status attn_common(const char* fn, const void* q, const void* k, cons
   if (err == nullptr) return fail(LVA_ERR_CUDA, "%s: cannot locate the device error word", fn);
   AttnArgs a{q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr,
              col_idx, col_len, mask_heads, scale, query_src, src_heads, err,
-             o_raster, T, Hg, Wg, tile_t, tile_h, tile_w, gather_windows, gather_window};
+             o_raster, T, Hg, Wg, tile_t, tile_h, tile_w, gather_windows, gather_window, lse_only};
   const char* why = "launch";
   cudaError_t e = launch_attn(a, stream, &why);
   if (e != cudaSuccess) return fail(LVA_ERR_CUDA, "%s: %s: %s", fn, why, cudaGetErrorString(e));
@@ -234,6 +257,15 @@ lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, vo
   return attn_common("attn", q, k, v, o, lse, B, H, n_pad, n_valid, d, block_size, row_ptr, col_idx,
                      col_len, mask_heads, scale, query_src, src_heads, nullptr, 0, 0, 0, 0, 0, 0, 0, 0,
                      stream);
+}
+
+lva_status lva_block_sparse_lse(const void* q, const void* k, float* lse, int B, int H, int64_t n_pad,
+                                int64_t n_valid, int d, int block_size, const int32_t* row_ptr,
+                                const int32_t* col_idx, int64_t col_len, int mask_heads, float scale,
+                                cudaStream_t stream) {
+  return attn_common("lse", q, k, nullptr, nullptr, lse, B, H, n_pad, n_valid, d, block_size, row_ptr,
+                     col_idx, col_len, mask_heads, scale, nullptr, 1, nullptr, 0, 0, 0, 0, 0, 0, 0, 0,
+                     stream, 1);
 }
 
 lva_status lva_block_sparse_attn_raster(const void* q, const void* k, const void* v, void* o_raster,
@@ -357,14 +389,18 @@ lva_status lva_device_error(cudaStream_t stream, lva_status* status, int* detail
   if (err == nullptr) return fail(LVA_ERR_CUDA, "device_error: cannot locate the device error word");
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return from_cuda(e, "device_error: stream sync");
-  int host[2] = {0, 0};
-  e = cudaMemcpy(host, err, sizeof(host), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return from_cuda(e, "device_error: read");
-  const int zero[2] = {0, 0};
-  e = cudaMemcpy(err, zero, sizeof(zero), cudaMemcpyHostToDevice);
-  if (e != cudaSuccess) return from_cuda(e, "device_error: clear");
-  *status = static_cast<lva_status>(host[0]);
-  if (detail) *detail = host[1];
+  unsigned long long word = 0;
+  {
+    std::lock_guard<std::mutex> lock(g_take_mutex);
+    take_error_kernel<<<1, 1, 0, stream>>>(reinterpret_cast<unsigned long long*>(err));
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return from_cuda(e, "device_error: exchange launch");
+    e = cudaMemcpyFromSymbolAsync(&word, g_device_error_taken, sizeof(word), 0, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return from_cuda(e, "device_error: read");
+  }
+  *status = static_cast<lva_status>(static_cast<int>(word & 0xffffffffull));
+  if (detail) *detail = static_cast<int>(word >> 32);
   return ok();
 }
 

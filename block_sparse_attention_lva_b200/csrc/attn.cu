@@ -25,6 +25,9 @@
 //                TMEM shapes), so row maxima and sums meet through one shuffle; O is
 //                rescaled in TMEM only when the running max grows by more than 2^8.
 //
+// The LSE-only form (lva_block_sparse_lse) runs the same roles without the V producer, the
+// P V issuer, the P stores and the O epilogue: its softmax only sums.
+//
 // Shared-memory operands use the 128-byte swizzle that TMA writes: a 64-element (128 B)
 // slice of each row, eight rows per 1024-byte atom.  Q and K are K-major; V is read
 // MN-major straight from its [keys, d] layout; P is the TMEM A operand of P*V.
@@ -38,20 +41,6 @@
 
 namespace lva {
 namespace {
-
-// Optional pipeline trace (compiled only with -DLVA_TRACE=<first CTA>): clock64 stamps of
-// pipeline events for kTraceCtas CTAs from the given one, slot = event * 64 + list position.
-#ifdef LVA_TRACE
-constexpr int kTraceCtas = 64, kTraceSlots = 32 * 64, kTraceBase = LVA_TRACE;
-__device__ unsigned long long g_trace[kTraceCtas][kTraceSlots];
-#define LVA_TRACE_AT(ev, t)                                                         \
-  do {                                                                              \
-    if (blockIdx.x >= kTraceBase && blockIdx.x < kTraceBase + kTraceCtas && (t) < 64) \
-      g_trace[blockIdx.x - kTraceBase][(ev) * 64 + (t)] = clock64();                   \
-  } while (0)
-#else
-#define LVA_TRACE_AT(ev, t) do { } while (0)
-#endif
 
 constexpr int BM = 128;            // query rows per MMA tile (TMEM lanes)
 constexpr int kSoftmaxWarp0 = 2;
@@ -82,9 +71,9 @@ struct AttnParams {
   int* err;
 };
 
-template <int D, int BN>
+template <int D, int BN, bool LSE_ONLY>
 struct Cfg {
-  static constexpr int KST = 3, VST = 3;
+  static constexpr int KST = 3, VST = LSE_ONLY ? 0 : 3;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int OFF_Q = 0;
@@ -111,9 +100,11 @@ struct Cfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
 };
 
-// The CSR row of a work item, checked so that no read or TMA coordinate leaves its buffer.
-// Called by every thread (whole warps); each warp checks the row cooperatively, so every
-// role reaches the same answer from the same memory.
+// The CSR row of a work item, checked so that no read or TMA coordinate leaves its buffer
+// and so that no key block is counted twice: the row must lie inside col_len and list
+// strictly ascending block indices in [0, nb).  Called by every thread (whole warps); each
+// warp checks the row cooperatively, so every role reaches the same answer from the same
+// memory.
 __device__ __forceinline__ int csr_row(const AttnParams& p, int64_t row, int32_t& start,
                                        bool& bad) {
   const int32_t a = __ldg(p.row_ptr + row), b = __ldg(p.row_ptr + row + 1);
@@ -123,7 +114,8 @@ __device__ __forceinline__ int csr_row(const AttnParams& p, int64_t row, int32_t
   bool lane_bad = false;
   for (int32_t t = a + int32_t(threadIdx.x & 31); t < b; t += 32) {
     const int32_t j = __ldg(p.col_idx + t);
-    lane_bad |= (j < 0 || j >= p.nb);
+    const int32_t prev = t > a ? __ldg(p.col_idx + t - 1) : -1;
+    lane_bad |= (j < 0 || j >= p.nb || j <= prev);
   }
   bad = __any_sync(0xffffffffu, lane_bad);
   if (bad) return 0;
@@ -131,11 +123,11 @@ __device__ __forceinline__ int csr_row(const AttnParams& p, int64_t row, int32_t
   return b - a;
 }
 
-template <int D, int BN, int KPC>
+template <int D, int BN, int KPC, bool LSE_ONLY>
 __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
-  using C = Cfg<D, BN>;
+  using C = Cfg<D, BN, LSE_ONLY>;
   // 128-byte-swizzled TMA tiles need 1024-byte aligned shared memory.
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t s_base = smem_u32(smem);
@@ -213,7 +205,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (threadIdx.x == 0) LVA_TRACE_AT(20, 0);
 
   // TMA load of the 64-element column chunk c of the rows [k0, k0 + box) of a plane:
   // plane-major rows, or (window-gather maps) row k = pos * m + a of the window-transposed
@@ -276,8 +267,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     produce(&tm_k, sK, C::KST, bar_k_full(0), bar_k_empty(0), 1, true);
   } else if (warp == kVWarp) {
     // ------------------------------------------------------------ TMA producer: V
-    if (lane == 0) tma_prefetch_desc(&tm_v);
-    produce(&tm_v, sV, C::VST, bar_v_full(0), bar_v_empty(0), 6, false);
+    if constexpr (!LSE_ONLY) {
+      if (lane == 0) tma_prefetch_desc(&tm_v);
+      produce(&tm_v, sV, C::VST, bar_v_full(0), bar_v_empty(0), 6, false);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer: S = Q K^T
     // S(T+2) is issued as soon as the softmax has read S(T) (same S buffer).  O += P V is
@@ -300,7 +293,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           if (!mbar_wait(bar_k_full(s), int(T / C::KST) & 1, abort_flag)) { ok = false; break; }
           if (T >= 2 && !mbar_wait(bar_s_free(b), int((T >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          LVA_TRACE_AT(0, nq == 0 ? t : 64);
           const uint64_t ks = k_desc + uint64_t((s * C::KV_BYTES) >> 4);
           const uint32_t s_tm = tmem + C::TM_S + 128 * b;
 #pragma unroll
@@ -327,44 +319,45 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       }
     }
   } else if (warp == kPVWarp) {
-    // ------------------------------------------------------------ MMA issuer: O += P V
-    // O += P(T) V_T as soon as P(T) is in TMEM and V_T has landed; P is the TMEM A operand.
-    // An item's first P V overwrites O, so it waits until the softmax warps have read the
-    // previous item's O in their epilogue.
-    const uint64_t v_desc = smem_desc_sw128(sV, BN * 128, 1024);
-    bool ok = true, any_mma = false;
-    uint32_t T = 0;
-    int nq = 0;
-    for (int it = it_begin; ok && it < it_end; ++it) {
-      const Item w = item_at(it);
-      if (w.n == 0) continue;
-      if (lane == 0) {
-        if (nq > 0) ok = mbar_wait(bar_o_free, (nq - 1) & 1, abort_flag);
-        for (int t = 0; ok && t < w.n; ++t, ++T) {
-          const int s = int(T % C::VST), b = int(T & 1);
-          if (!mbar_wait(bar_p_full(b), int(T >> 1) & 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(bar_v_full(s), int(T / C::VST) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          LVA_TRACE_AT(1, nq == 0 ? t : 64);
-          const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
-          const uint32_t p_tm = tmem + C::TM_P + 64 * b;
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            umma_f16_ts(tmem + C::TM_O, p_tm + kk * 8, vs + uint64_t((kk * 16 * 128) >> 4), C::IDESC_PV,
-                        (t > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(bar_v_empty(s));
-          umma_commit(bar_o_done(b));
-          any_mma = true;
+    if constexpr (!LSE_ONLY) {
+      // ------------------------------------------------------------ MMA issuer: O += P V
+      // O += P(T) V_T as soon as P(T) is in TMEM and V_T has landed; P is the TMEM A operand.
+      // An item's first P V overwrites O, so it waits until the softmax warps have read the
+      // previous item's O in their epilogue.
+      const uint64_t v_desc = smem_desc_sw128(sV, BN * 128, 1024);
+      bool ok = true, any_mma = false;
+      uint32_t T = 0;
+      int nq = 0;
+      for (int it = it_begin; ok && it < it_end; ++it) {
+        const Item w = item_at(it);
+        if (w.n == 0) continue;
+        if (lane == 0) {
+          if (nq > 0) ok = mbar_wait(bar_o_free, (nq - 1) & 1, abort_flag);
+          for (int t = 0; ok && t < w.n; ++t, ++T) {
+            const int s = int(T % C::VST), b = int(T & 1);
+            if (!mbar_wait(bar_p_full(b), int(T >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(bar_v_full(s), int(T / C::VST) & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
+            const uint32_t p_tm = tmem + C::TM_P + 64 * b;
+  #pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              umma_f16_ts(tmem + C::TM_O, p_tm + kk * 8, vs + uint64_t((kk * 16 * 128) >> 4), C::IDESC_PV,
+                          (t > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(bar_v_empty(s));
+            umma_commit(bar_o_done(b));
+            any_mma = true;
+          }
+          ++nq;
         }
-        ++nq;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
       }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-    }
-    if (lane == 0) {
-      if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 7); }
-      if (any_mma) {
-        umma_commit(bar_final_pv);
-        mbar_wait(bar_final_pv, 0, never);
+      if (lane == 0) {
+        if (!ok) { *abort_flag = 1; report_fault(p.err, 5, 7); }
+        if (any_mma) {
+          umma_commit(bar_final_pv);
+          mbar_wait(bar_final_pv, 0, never);
+        }
       }
     }
   } else {
@@ -380,7 +373,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     const uint32_t lane_off = uint32_t(quarter * 32 + sel * 16) << 16;
     const float c = p.scale_log2;                 // scores -> log2 units
     bool ok = true;
-    const bool tr = (quarter == 2 && sel == 0 && lane == 0);
     uint32_t T = 0;
     int nq = 0;
     for (int it = it_begin; ok && it < it_end; ++it) {
@@ -399,7 +391,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         if (t + 1 < n) jn = __ldg(p.col_idx + w.start + t + 1);
         if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T >> 1) & 1, abort_flag))) { ok = false; break; }
         tc_fence_after();
-        if (tr && nq == 0) LVA_TRACE_AT(2, t);
         uint32_t sr[HALF];
 #pragma unroll
         for (int q = 0; q < HALF / 32; ++q)
@@ -409,7 +400,6 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_s_free(b));
-        if (tr && nq == 0) LVA_TRACE_AT(3, t);
         // Real keys of this half (only the block holding the sequence end is partial).  The
         // choice of path is made for the whole warp: the exponential loop below issues
         // warp-collective TMEM stores, and the two halves of a row can differ at the end.
@@ -449,7 +439,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         // P_b was last read by O += P(t-2) V; wait for it before any part of P(t) is stored.
         // Each P buffer has its own completion barrier, so the wait never aliases an older
         // phase.  (Almost always complete by now: P(t-2) V was issued a block earlier.)
-        if (T >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), int((T >> 1) - 1) & 1, abort_flag))) {
+        if (!LSE_ONLY && T >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), int((T >> 1) - 1) & 1, abort_flag))) {
           ok = false; break;
         }
         tc_fence_after();
@@ -475,17 +466,21 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
               p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
             }
             acc[e & 1] = f2_add(acc[e & 1], p2);
-            float p0, p1;
-            f2_unpack(p2, p0, p1);
-            pk[e] = pack_bf16x2(p0, p1);
-            if constexpr (HALF == 64) {
-              if (e == 15) tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+            if constexpr (!LSE_ONLY) {
+              float p0, p1;
+              f2_unpack(p2, p0, p1);
+              pk[e] = pack_bf16x2(p0, p1);
+              if constexpr (HALF == 64) {
+                if (e == 15) tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+              }
             }
           }
-          if constexpr (HALF == 64) {
-            tmem_st_16x2_16<HALF / 2>(p_tm + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
-          } else {
-            tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          if constexpr (!LSE_ONLY) {
+            if constexpr (HALF == 64) {
+              tmem_st_16x2_16<HALF / 2>(p_tm + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
+            } else {
+              tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+            }
           }
           float a0, a1, b0, b1;
           f2_unpack(acc[0], a0, a1);
@@ -500,23 +495,22 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
             pk[e / 2] = pack_bf16x2(p0, p1);
           }
           // P half row (bf16 pairs) -> TMEM P_b, the A operand of O += P V.
-          if constexpr (HALF == 64) {
+          if constexpr (LSE_ONLY) {
+          } else if constexpr (HALF == 64) {
             tmem_st_16x2_32<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[32]>(pk));
           } else {
             tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
           }
         }
         l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
-        if (tr && nq == 0) LVA_TRACE_AT(4, t);
 
         // O was last written by O += P(t-1) V: rescale it (rarely) once that has completed,
         // before P(t) is released to the P V issuer.
-        if (t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if (!LSE_ONLY && t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
           if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(b ^ 1), int((T - 1) >> 1) & 1, abort_flag))) {
             ok = false; break;
           }
           tc_fence_after();
-          if (tr && nq == 0) LVA_TRACE_AT(5, t);
   #pragma unroll 1
           for (int q = 0; q < DH / 32; ++q) {
             uint32_t ov[32];
@@ -527,11 +521,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
             tmem_st_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
           }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_p_full(b));
-        if (tr && nq == 0) LVA_TRACE_AT(7, t);
+        if constexpr (!LSE_ONLY) {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_p_full(b));
+        }
       }
       if (!ok) break;
 
@@ -540,49 +535,51 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       const int i = w.i;
       const int64_t grow = int64_t(i) * BN + row;           // row within the plane
       const bool store = row < BN && grow < p.n_pad;
-      // O row destination: tile order, or (fused inverse reorder) the row's raster position;
-      // padding rows have no raster position and are not written then.
-      __nv_bfloat16* orow;
-      bool store_o = store;
-      if (p.o_raster != nullptr) {
-        store_o = store && grow < p.n_valid;
-        const uint32_t raster = store_o ? tile_order_to_raster(uint32_t(grow), p.grid) : 0u;
-        orow = p.o_raster + (plane * p.n_valid + int64_t(raster)) * D + hf * DH;
-      } else {
-        orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
-      }
       const float l_row = l + __shfl_xor_sync(0xffffffffu, l, 16);
       const bool have = n > 0 && l_row > 0.f;
-      const float inv_l = have ? 1.f / l_row : 0.f;
-      if (n > 0) {
-        const uint32_t T_last = T - 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(int(T_last & 1)), int(T_last >> 1) & 1, abort_flag))) {
-          ok = false; break;
+      if constexpr (!LSE_ONLY) {
+        // O row destination: tile order, or (fused inverse reorder) the row's raster position;
+        // padding rows have no raster position and are not written then.
+        __nv_bfloat16* orow;
+        bool store_o = store;
+        if (p.o_raster != nullptr) {
+          store_o = store && grow < p.n_valid;
+          const uint32_t raster = store_o ? tile_order_to_raster(uint32_t(grow), p.grid) : 0u;
+          orow = p.o_raster + (plane * p.n_valid + int64_t(raster)) * D + hf * DH;
+        } else {
+          orow = p.o + (plane * p.n_pad + grow) * D + hf * DH;
         }
-        tc_fence_after();
-      }
-#pragma unroll 1
-      for (int q = 0; q < DH / 32; ++q) {
-        uint32_t ov[32];
+        const float inv_l = have ? 1.f / l_row : 0.f;
         if (n > 0) {
-          tmem_ld_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
-          tmem_wait_ld();
-          if (q == DH / 32 - 1) {
-            // All of O is in registers: the next item's first P V may overwrite it.
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_o_free);
+          const uint32_t T_last = T - 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(int(T_last & 1)), int(T_last >> 1) & 1, abort_flag))) {
+            ok = false; break;
           }
+          tc_fence_after();
         }
-        if (store_o) {
-#pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w4[e] = have ? pack_bf16x2(__uint_as_float(ov[8 * e4 + 2 * e]) * inv_l,
-                                         __uint_as_float(ov[8 * e4 + 2 * e + 1]) * inv_l) : 0u;
-            reinterpret_cast<uint4*>(orow + q * 32)[e4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  #pragma unroll 1
+        for (int q = 0; q < DH / 32; ++q) {
+          uint32_t ov[32];
+          if (n > 0) {
+            tmem_ld_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
+            tmem_wait_ld();
+            if (q == DH / 32 - 1) {
+              // All of O is in registers: the next item's first P V may overwrite it.
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(bar_o_free);
+            }
+          }
+          if (store_o) {
+  #pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) {
+              uint32_t w4[4];
+  #pragma unroll
+              for (int e = 0; e < 4; ++e)
+                w4[e] = have ? pack_bf16x2(__uint_as_float(ov[8 * e4 + 2 * e]) * inv_l,
+                                           __uint_as_float(ov[8 * e4 + 2 * e + 1]) * inv_l) : 0u;
+              reinterpret_cast<uint4*>(orow + q * 32)[e4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
           }
         }
       }
@@ -601,20 +598,20 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   }
 }
 
-template <int D, int BN, int KPC>
+template <int D, int BN, int KPC, bool LSE_ONLY>
 cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why) {
-  using C = Cfg<D, BN>;
+  using C = Cfg<D, BN, LSE_ONLY>;
   const int64_t rows = int64_t(a.B) * a.H * a.n_pad;
   CUtensorMap tq, tk, tv;
   bool maps_ok;
   if (a.gather_windows == 0) {
     maps_ok = make_rows_map(&tq, a.q, rows, D, BM) && make_rows_map(&tk, a.k, rows, D, BN) &&
-              make_rows_map(&tv, a.v, rows, D, BN);
+              make_rows_map(&tv, LSE_ONLY ? a.k : a.v, rows, D, BN);
   } else {
     const int64_t planes = int64_t(a.B) * a.H;
     maps_ok = make_window_gather_map(&tq, a.q, planes, a.gather_windows, a.gather_window, D, BM) &&
               make_window_gather_map(&tk, a.k, planes, a.gather_windows, a.gather_window, D, BN) &&
-              make_window_gather_map(&tv, a.v, planes, a.gather_windows, a.gather_window, D, BN);
+              make_window_gather_map(&tv, LSE_ONLY ? a.k : a.v, planes, a.gather_windows, a.gather_window, D, BN);
   }
   if (!maps_ok) {
     *why = "cuTensorMapEncodeTiled failed or is unavailable";
@@ -622,7 +619,7 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   }
   static DeviceFlags attr_set = {};
   cudaError_t e = once_per_device(attr_set, [] {
-    return cudaFuncSetAttribute(bsa_fwd_kernel<D, BN, KPC>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(bsa_fwd_kernel<D, BN, KPC, LSE_ONLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 C::SMEM_BYTES);
   });
   if (e != cudaSuccess) { *why = "cudaFuncSetAttribute(max dynamic smem) failed"; return e; }
@@ -649,17 +646,11 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   if (items == 0) return cudaSuccess;
   p.items = items;
   const int64_t grid = (items + KPC - 1) / KPC;
-  bsa_fwd_kernel<D, BN, KPC><<<dim3(unsigned(grid)), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  bsa_fwd_kernel<D, BN, KPC, LSE_ONLY><<<dim3(unsigned(grid)), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
 }  // namespace
-
-#ifdef LVA_TRACE
-extern "C" int lva_trace_copy(void* dst, size_t bytes) {
-  return int(cudaMemcpyFromSymbol(dst, g_trace, bytes < sizeof(g_trace) ? bytes : sizeof(g_trace)));
-}
-#endif
 
 // Query blocks per CTA.  A CTA walks a run of consecutive query blocks: its prologue
 // (barriers, TMEM allocation, the first Q and K tiles) is paid once per run and the next
@@ -668,19 +659,27 @@ extern "C" int lva_trace_copy(void* dst, size_t bytes) {
 // query block) and costs tail balance and L2 locality for long ones.  With col_len taken as
 // the entry count: runs of 8 for rows averaging at most 3 key blocks, 4 for at most 8,
 // otherwise 1 (a capacity larger than the entry count therefore selects 1).
-template <int D, int BN>
+template <int D, int BN, bool LSE_ONLY>
 cudaError_t launch_dispatch(const AttnArgs& a, cudaStream_t stream, const char** why) {
   const int64_t rows = int64_t(a.mask_heads) * (a.n_pad / a.block_size);
-  if (rows > 0 && a.col_len <= 3 * rows) return launch_cfg<D, BN, 8>(a, stream, why);
-  if (rows > 0 && a.col_len <= 8 * rows) return launch_cfg<D, BN, 4>(a, stream, why);
-  return launch_cfg<D, BN, 1>(a, stream, why);
+  if (rows > 0 && a.col_len <= 3 * rows) return launch_cfg<D, BN, 8, LSE_ONLY>(a, stream, why);
+  if (rows > 0 && a.col_len <= 8 * rows) return launch_cfg<D, BN, 4, LSE_ONLY>(a, stream, why);
+  return launch_cfg<D, BN, 1, LSE_ONLY>(a, stream, why);
 }
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why) {
-  if (a.d == 128 && a.block_size == 128) return launch_dispatch<128, 128>(a, stream, why);
-  if (a.d == 128 && a.block_size == 64) return launch_dispatch<128, 64>(a, stream, why);
-  if (a.d == 64 && a.block_size == 128) return launch_dispatch<64, 128>(a, stream, why);
-  if (a.d == 64 && a.block_size == 64) return launch_dispatch<64, 64>(a, stream, why);
+  if (a.lse_only) {
+    // LSE only (lva_block_sparse_lse): no V, no P V product, no O
+    if (a.d == 128 && a.block_size == 128) return launch_dispatch<128, 128, true>(a, stream, why);
+    if (a.d == 128 && a.block_size == 64) return launch_dispatch<128, 64, true>(a, stream, why);
+    if (a.d == 64 && a.block_size == 128) return launch_dispatch<64, 128, true>(a, stream, why);
+    if (a.d == 64 && a.block_size == 64) return launch_dispatch<64, 64, true>(a, stream, why);
+  } else {
+    if (a.d == 128 && a.block_size == 128) return launch_dispatch<128, 128, false>(a, stream, why);
+    if (a.d == 128 && a.block_size == 64) return launch_dispatch<128, 64, false>(a, stream, why);
+    if (a.d == 64 && a.block_size == 128) return launch_dispatch<64, 128, false>(a, stream, why);
+    if (a.d == 64 && a.block_size == 64) return launch_dispatch<64, 64, false>(a, stream, why);
+  }
   *why = "unsupported (d, block_size)";
   return cudaErrorInvalidValue;
 }

@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(kEThreads, 2) block_energy_kernel(
     bool lane_bad = false;
     for (int32_t t = a + lane; t < b_end; t += 32) {
       const int32_t j = __ldg(p.col_idx + t);
-      lane_bad |= (j < 0 || j >= p.nb);
+      const int32_t prev = t > a ? __ldg(p.col_idx + t - 1) : -1;
+      lane_bad |= (j < 0 || j >= p.nb || j <= prev);   // in range, strictly ascending
     }
     bad = __any_sync(0xffffffffu, lane_bad);
   }

@@ -8,6 +8,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "lva.h"
+
 namespace lva {
 
 // Per-device setup done once (a kernel's shared-memory limit, a looked-up attribute).  The
@@ -75,6 +77,7 @@ struct AttnArgs {
   int T, Hg, Wg, tt, th, tw; // latent grid and tile (used with o_raster)
   int gather_windows;        // 0, or m: q, k, v are read window-transposed (see api.cu)
   int gather_window;         // w, the tokens per window, with gather_windows
+  int lse_only;              // 1: only LSE is computed (v, o and o_raster unused)
 };
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why);
 
@@ -142,6 +145,10 @@ bool make_window_gather_map(CUtensorMap* m, const void* base, int64_t planes, in
 
 // Device error word of the current device (from api.cu).
 int* device_error_word();
+
+// Sets the calling thread's lva_last_error_message (printf-style) and returns `status`
+// (from api.cu; an empty message for LVA_OK).
+lva_status set_error_message(lva_status status, const char* fmt, ...);
 
 // Bounded-wait self-test (selftest.cu): mode 0 = nothing arrives, 1 = abort flag raised,
 // 2 = the peer arrives.

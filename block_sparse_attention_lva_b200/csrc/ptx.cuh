@@ -11,11 +11,15 @@
 
 namespace lva {
 
-// Kernel-side error word: [0] = lva_status of the first fault, [1] = detail code.
-// Written with atomicCAS so the first fault wins.
+// Kernel-side error word: [0] = lva_status of the first fault, [1] = detail code, as one
+// 8-byte-aligned 64-bit word (status in the low half).  Both halves are written by one
+// compare-and-swap from zero, so the first fault wins and a reader never sees a status
+// paired with another fault's detail.
 __device__ __forceinline__ void report_fault(int* err, int status, int detail) {
-  if (err != nullptr && atomicCAS(err, 0, status) == 0) {
-    atomicExch(err + 1, detail);
+  if (err != nullptr) {
+    const unsigned long long v =
+        (static_cast<unsigned long long>(static_cast<uint32_t>(detail)) << 32) | static_cast<uint32_t>(status);
+    atomicCAS(reinterpret_cast<unsigned long long*>(err), 0ull, v);
   }
 }
 
@@ -89,9 +93,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Same contract as mbar_wait, but lets the thread sleep inside mbarrier.try_wait between
-// polls: for waits whose latency is off the critical path (it frees issue slots for the
-// warps that share the scheduler).
+// Same contract as mbar_wait, but waits inside mbarrier.try_wait, which suspends the thread
+// until the phase completes (or a system-dependent time limit passes): a waiting warp takes
+// no issue slots from the warps that share its scheduler, which matters when two CTAs share
+// an SM and one CTA's warps wait while the other's compute.
 __device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();

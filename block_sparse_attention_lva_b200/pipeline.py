@@ -14,6 +14,8 @@ need the tile-order broadcast between them.
 """
 from __future__ import annotations
 
+import ctypes
+
 import torch
 
 from . import _binding as lb
@@ -169,16 +171,14 @@ class VideoBlockSparseAttention:
 
 
     def forward_host(self, qkv_host, o_host, lse_host, step: int = 0, chunks: int = 6, wait: bool = True):
-        """One layer step from and to pinned host memory, with the copies overlapped.
+        """One layer step from and to pinned host memory, through ``lva_layer_step_host``.
 
         ``qkv_host``: pinned bf16 [3, B, H, N, d] (raster Q, K, V); ``o_host``: pinned bf16
         [B, H, N, d] (raster O, written); ``lse_host``: pinned fp32 [B, H, n_pad] (tile-order
-        LSE, written).  Heads are independent given the mask, so the step runs per group of
-        heads of one batch element: the host-to-device copy of group c+1 and the
-        device-to-host copy of group c-1 proceed while group c is reordered and attended.
-        Consecutive calls overlap too: the device staging and output buffers are
-        double-buffered, so a call's host-to-device copies start while the previous call is
-        still computing and copying back.
+        LSE, written).  The C call runs the step per group of heads (about ``chunks`` groups),
+        with each group's host-to-device copy, compute and device-to-host copy on three
+        streams, so one group's copies overlap the others' compute.  Two device buffer sets
+        (staging, outputs, events) are used alternately, so consecutive calls overlap as well.
 
         Returns a CUDA event that completes when ``o_host`` and ``lse_host`` hold this step's
         results; the host buffers must not be rewritten or read before then.  With ``wait``
@@ -195,88 +195,41 @@ class VideoBlockSparseAttention:
         for name, t, _, _ in bufs:
             if not t.is_pinned():
                 raise ValueError(f"{name} must be in pinned host memory (copies overlap compute)")
+        cur = torch.cuda.current_stream(self.device)
         if not hasattr(self, "_host_io"):
             mk = lambda shape, dt: torch.empty(shape, dtype=dt, device=self.device)
-            self._host_io = dict(
-                qkv=[mk((3, B, H, N, d), torch.bfloat16) for _ in range(2)],
-                o=[mk((B, H, N, d), torch.bfloat16) for _ in range(2)],
-                lse=[mk((B, H, self.n_pad), torch.float32) for _ in range(2)],
-                staging_free=[None, None], out_free=[None, None], computed=None, slot=0,
-                h2d=torch.cuda.Stream(self.device), d2h=torch.cuda.Stream(self.device))
+            groups = B * -(-H // -(-H // max(1, min(H, -(-chunks // B)))))
+            sets = []
+            for _ in range(2):
+                events = [torch.cuda.Event() for _ in range(2 * groups + 2)]
+                for ev in events:                 # creates the CUDA events (a no-op on the stream)
+                    ev.record(cur)
+                arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+                t = dict(qkv=mk((3, B, H, N, d), torch.bfloat16), o=mk((B, H, N, d), torch.bfloat16),
+                         lse=mk((B, H, self.n_pad), torch.float32), events=events, arr=arr)
+                t["c"] = lb.LvaHostStepBuffers(
+                    t["qkv"].data_ptr(), t["o"].data_ptr(), t["lse"].data_ptr(), self.qkv_t.data_ptr(),
+                    self.o_t.data_ptr(), self.row_ptr.data_ptr(), self.col_idx.data_ptr(), self.col_idx.numel(),
+                    self.col_idx.numel(), self.nnz.data_ptr(), arr, len(events))
+                sets.append(t)
+            self._host_io = dict(sets=sets, slot=0, chunks=chunks,
+                                 h2d=torch.cuda.Stream(self.device), d2h=torch.cuda.Stream(self.device),
+                                 shape=lb.LvaLayerShape(B, H, d, self.block_size, *self.grid, *self.tile, self.scale))
         io = self._host_io
-        sl = io["slot"]
-        io["slot"] = sl ^ 1
-        qkv_dev, o_dev, lse_dev = io["qkv"][sl], io["o"][sl], io["lse"][sl]
-        s_h2d, s_d2h = io["h2d"], io["d2h"]
-        cur = torch.cuda.current_stream(self.device)
-        groups = []
-        per = max(1, -(-H // max(1, chunks // max(1, B))))
-        for b in range(B):
-            for h0 in range(0, H, per):
-                groups.append((b, h0, min(H, h0 + per)))
-        # Host-to-device: staging slot `sl` was last read by the compute of two calls ago.
-        if io["staging_free"][sl] is not None:
-            s_h2d.wait_event(io["staging_free"][sl])
-        in_ready, out_ready = [], []
-        for b, h0, h1 in groups:
-            with torch.cuda.stream(s_h2d):
-                for t in range(3):
-                    qkv_dev[t, b, h0:h1].copy_(qkv_host[t, b, h0:h1], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(s_h2d)
-            in_ready.append(ev)
-        # Output slot `sl` was last read by the copies back of two calls ago; the tile-order
-        # buffers and the CSR are shared by all calls, so the mask build and the compute also
-        # follow the previous call's compute (a no-op when the caller keeps one stream).
-        if io["out_free"][sl] is not None:
-            cur.wait_event(io["out_free"][sl])
-        if io["computed"] is not None:
-            cur.wait_event(io["computed"])
+        if chunks != io["chunks"]:
+            raise ValueError(f"chunks is fixed at the first call ({io['chunks']})")
+        t = io["sets"][io["slot"]]
+        io["slot"] ^= 1
+        # The CSR for this step (built on the current stream, which also runs the step's
+        # compute); the C call then uses it as it stands.
         self.build_mask(step)
-        # The static-mask and repetitive-head tables are indexed per head of the group.
-        nb = self.nb
-        for (b, h0, h1), ev in zip(groups, in_ready):
-            cur.wait_event(ev)
-            hn = h1 - h0
-            P = hn
-            for t, dst in ((0, self.q_t), (1, self.k_t), (2, self.v_t)):
-                lb.lva_reorder_tokens(qkv_dev[t, b, h0:h1].reshape(P, N, d),
-                                      dst[b, h0:h1].reshape(P, self.n_pad, d), self.grid, self.tile,
-                                      self.n_pad, inverse=False)
-            mh = self.mask_heads
-            row_ptr = self.row_ptr if mh == 1 else self.row_ptr[h0 * nb:]
-            qkv_t = (self.q_t[b:b + 1, h0:h1], self.k_t[b:b + 1, h0:h1], self.v_t[b:b + 1, h0:h1])
-            if self.query_src is None:
-                lb.lva_block_sparse_attn_raster(*qkv_t, o_dev[b:b + 1, h0:h1], lse_dev[b:b + 1, h0:h1], N,
-                                                self.block_size, row_ptr, self.col_view, 1 if mh == 1 else hn,
-                                                self.scale, self.grid, self.tile)
-            else:
-                qs = self.query_src if self.query_src.shape[0] == 1 else self.query_src[h0:h1]
-                lb.lva_block_sparse_attn(*qkv_t, self.o_t[b:b + 1, h0:h1], lse_dev[b:b + 1, h0:h1], N,
-                                         self.block_size, row_ptr, self.col_view, 1 if mh == 1 else hn,
-                                         self.scale, qs)
-                lb.lva_broadcast_blocks(self.o_t[b:b + 1, h0:h1], lse_dev[b:b + 1, h0:h1], self.block_size, qs)
-                lb.lva_reorder_tokens(self.o_t[b, h0:h1].reshape(P, self.n_pad, d),
-                                      o_dev[b, h0:h1].reshape(P, N, d), self.grid, self.tile, self.n_pad,
-                                      inverse=True)
-            ev = torch.cuda.Event()
-            ev.record(cur)
-            out_ready.append(ev)
-        staging_free = torch.cuda.Event()
-        staging_free.record(cur)
-        io["staging_free"][sl] = staging_free
-        io["computed"] = staging_free
-        for (b, h0, h1), ev in zip(groups, out_ready):
-            s_d2h.wait_event(ev)
-            with torch.cuda.stream(s_d2h):
-                o_host[b, h0:h1].copy_(o_dev[b, h0:h1], non_blocking=True)
-                lse_host[b, h0:h1].copy_(lse_dev[b, h0:h1], non_blocking=True)
-        done = torch.cuda.Event()
-        done.record(s_d2h)
-        io["out_free"][sl] = done
+        t["c"].col_len = self.col_view.numel()
+        done = lb.lva_layer_step_host(qkv_host, o_host, lse_host, io["shape"], self.params, self.dense_mask,
+                                      False, self.query_src, t["c"], chunks, io["h2d"], io["d2h"], cur)
+        ev = next(e for e in t["events"] if e.cuda_event == done)
         if wait:
-            cur.wait_event(done)
-        return done
+            cur.wait_event(ev)
+        return ev
 
 
 class SquadTwoPass:
@@ -340,7 +293,8 @@ class StaticMaskCalibrator:
     one batch element of one ``add_prompt`` call) goes through
 
     1. ``lva_reorder_tokens`` of Q and K into tile order;
-    2. ``lva_block_sparse_attn`` with the all-ones mask, for the row LSE of dense attention;
+    2. ``lva_block_sparse_lse`` with the all-ones mask, for the row LSE of dense attention
+       (the attention kernel's scores, maxima and sums, with no V, P V product or O);
     3. ``lva_block_energy`` -> E [B, H, nb, nb], the attention mass of every block pair;
     4. ``lva_select_blocks`` with the timestep's threshold ``eps`` -> a 0/1 mask per sample;
 
@@ -361,7 +315,6 @@ class StaticMaskCalibrator:
         shape = (B, H, self.n_pad, d)
         self.qk_t = torch.empty((2,) + shape, dtype=torch.bfloat16, **kw)
         self.q_t, self.k_t = self.qk_t[0], self.qk_t[1]
-        self.o_t = torch.empty(shape, dtype=torch.bfloat16, **kw)     # dense-pass output, unused
         self.lse = torch.empty((B, H, self.n_pad), dtype=torch.float32, **kw)
         self.energy = torch.empty((B, H, self.nb, self.nb), dtype=torch.float32, **kw)
         p = lb.MaskParams(lb.LVA_MASK_ALL, self.n_pad, self.n_valid, block_size, 1)
@@ -377,9 +330,8 @@ class StaticMaskCalibrator:
         for src, dst in ((q, self.q_t), (k, self.k_t)):
             lb.lva_reorder_tokens(src.reshape(P, self.n_valid, self.d), dst.view(P, self.n_pad, self.d),
                                   self.grid, self.tile, self.n_pad, inverse=False)
-        # V only feeds the unused dense output; K stands in for it.
-        lb.lva_block_sparse_attn(self.q_t, self.k_t, self.k_t, self.o_t, self.lse, self.n_valid,
-                                 self.block_size, self.row_ptr, self.col_idx, 1, self.scale)
+        lb.lva_block_sparse_lse(self.q_t, self.k_t, self.lse, self.n_valid, self.block_size, self.row_ptr,
+                                self.col_idx, 1, self.scale)
         lb.lva_block_energy(self.q_t, self.k_t, self.lse, self.energy, self.n_valid, self.block_size,
                             self.row_ptr, self.col_idx, 1, self.scale)
         return self.energy

@@ -170,8 +170,10 @@ lva_status lva_build_block_mask(const lva_mask_params* params, const uint8_t* de
  *
  * q, k, v, o: device bf16 [B, H, n_pad, d], 16-byte aligned.  lse: device fp32 [B, H, n_pad].
  * row_ptr: device [mask_heads*nb + 1]; col_idx: device, col_len entries (the kernel never
- * reads past col_len; CSR entries out of range are skipped and reported through
- * lva_device_error as LVA_ERR_INVALID_ARG).  col_len may be the capacity of col_idx or the
+ * reads past col_len).  A CSR row that reaches outside [0, col_len), lists a block outside
+ * [0, nb) or does not list strictly ascending blocks is skipped (its query rows get O = 0,
+ * LSE = -inf) and reported through lva_device_error as LVA_ERR_INVALID_ARG (detail = the
+ * CSR row), so no key block is ever counted twice.  col_len may be the capacity of col_idx or the
  * exact entry count; the exact count lets the call see short rows, for which each CTA then
  * processes a run of consecutive query blocks (8 when rows average at most 3 key blocks, 4
  * when at most 8; results are identical either way).
@@ -186,6 +188,26 @@ lva_status lva_block_sparse_attn(const void* q, const void* k, const void* v, vo
                                  int block_size, const int32_t* row_ptr, const int32_t* col_idx,
                                  int64_t col_len, int mask_heads, float scale,
                                  const int32_t* query_src, int src_heads, cudaStream_t stream);
+
+/*
+ * lva_block_sparse_lse -- the row log-sum-exp of block-sparse attention, without O.
+ *
+ * The CalibAtt page ("Accelerating Text-to-Video Generation with Calibrated Sparse
+ * Attention", section 2 A.1) normalises the attention scores of every query row before
+ * summing them per block; with the all-ones block list this call gives that normaliser,
+ * LSE_r = m + ln(l) of lva_block_sparse_attn, for lva_block_energy.  It runs the same
+ * scores, maxima and sums in the same arithmetic as lva_block_sparse_attn (so the LSE is
+ * the one that call returns, up to the order of floating-point additions), but never loads
+ * V and computes no P V product and no O.
+ *
+ * q, k: device bf16 [B, H, n_pad, d], 16-byte aligned; lse: device fp32 [B, H, n_pad]
+ * (written).  CSR arguments, support and errors as for lva_block_sparse_attn (no
+ * repetitive-head maps).
+ */
+lva_status lva_block_sparse_lse(const void* q, const void* k, float* lse, int B, int H, int64_t n_pad,
+                                int64_t n_valid, int d, int block_size, const int32_t* row_ptr,
+                                const int32_t* col_idx, int64_t col_len, int mask_heads, float scale,
+                                cudaStream_t stream);
 
 /*
  * lva_block_sparse_attn_raster -- lva_block_sparse_attn with O written in raster order.
@@ -273,8 +295,9 @@ lva_status lva_broadcast_blocks(void* o, float* lse, int B, int H, int64_t n_pad
  * q, k: device bf16 [B, H, n_pad, d], 16-byte aligned; lse: device fp32 [B, H, n_pad];
  * energy: device fp32 [B, H, nb, nb] (caller-owned, written).  row_ptr / col_idx / col_len /
  * mask_heads: a CSR block list as for lva_block_sparse_attn (the all-ones list for a dense
- * calibration pass).  Bad CSR rows are skipped (their energy row stays 0) and reported
- * through lva_device_error as LVA_ERR_INVALID_ARG.
+ * calibration pass).  Bad CSR rows (outside col_len, a block outside [0, nb), or blocks not
+ * strictly ascending) are skipped (their energy row stays 0) and reported through
+ * lva_device_error as LVA_ERR_INVALID_ARG.
  * Supported: d in {64, 128}, block_size in {64, 128}, B*H*n_pad < 2^31.
  */
 lva_status lva_block_energy(const void* q, const void* k, const float* lse, float* energy, int B,
@@ -317,13 +340,85 @@ lva_status lva_select_blocks(const float* energy, uint8_t* mask, int64_t rows, i
 lva_status lva_aggregate_masks(const uint8_t* masks, uint8_t* out, int prompts, int64_t count,
                                double rho, cudaStream_t stream);
 
+/* Shape of one attention layer over a T x Hg x Wg latent grid (lva_layer_step_host). */
+typedef struct {
+  int B, H;                    /* batch elements and heads */
+  int d;                       /* head dim: 64 or 128 */
+  int block_size;              /* 64 or 128 */
+  int T, Hg, Wg;               /* latent grid: N = T*Hg*Wg tokens */
+  int tile_t, tile_h, tile_w;  /* tiles of the token order (lva_reorder_tokens) */
+  float scale;                 /* softmax scale, e.g. 1/sqrt(d) */
+} lva_layer_shape;
+
+/* Device buffers and events of lva_layer_step_host, all owned by the caller.  With
+ * n_pad = N rounded up to block_size and nb = n_pad / block_size: */
+typedef struct {
+  void* qkv_stage;      /* device bf16 [3, B, H, N, d]: the step's raster Q, K, V */
+  void* o_stage;        /* device bf16 [B, H, N, d]: the step's raster O */
+  float* lse_stage;     /* device fp32 [B, H, n_pad]: the step's LSE (tile order) */
+  void* qkv_tile;       /* device bf16 [3, B, H, n_pad, d]: Q, K, V in tile order */
+  void* o_tile;         /* device bf16 [B, H, n_pad, d]: O in tile order; only with query_src */
+  int32_t* row_ptr;     /* device int32 [mask_heads*nb + 1] */
+  int32_t* col_idx;     /* device int32 [col_capacity] */
+  int64_t col_capacity;
+  int64_t col_len;      /* CSR entries the attention may read: col_capacity, or the exact entry
+                           count when known (short rows then run several blocks per CTA) */
+  int32_t* nnz;         /* device int32 [1] */
+  cudaEvent_t* events;  /* num_events caller-created events, at least 2*groups + 2 */
+  int num_events;
+} lva_host_step_buffers;
+
+/*
+ * lva_layer_step_host -- one attention layer from and to pinned host memory.
+ *
+ * The layer step of the LVSA page ("LVSA: Training-Free Sparse Attention for Long Video
+ * Diffusion", technical summary section 2) and of the CalibAtt page ("Accelerating
+ * Text-to-Video Generation with Calibrated Sparse Attention", section 2 B) for inputs that
+ * live in host memory: for every batch element and group of heads,
+ *   copy raster Q, K, V in -> lva_reorder_tokens -> lva_block_sparse_attn_raster -> copy O
+ *   and LSE out,
+ * with the CSR of the step's mask built once first (lva_build_block_mask with `mask`, when
+ * build_mask != 0; otherwise row_ptr / col_idx must already hold it).  With query_src (the
+ * repetitive heads of lva_block_sparse_attn) a group runs lva_block_sparse_attn into o_tile,
+ * lva_broadcast_blocks and the inverse lva_reorder_tokens instead.  The results are those
+ * of the same calls on device buffers, bit for bit.
+ *
+ * Heads are split into up to ceil(head_groups / B) groups per batch element (runs of
+ * ceil(H / groups) heads).  Each group's three input copies (one cudaMemcpyAsync each) go on
+ * `h2d`, its compute on `compute` and its two output copies on `d2h`, ordered by the events
+ * of `bufs`, so one group's copies overlap the others' compute.  Two buffer sets (each with
+ * its own staging, outputs and events; the tile-order and CSR buffers may be shared) used
+ * alternately let consecutive steps overlap as well: a step waits only for the previous use
+ * of its own buffer set.
+ *
+ * qkv_host: pinned bf16 [3, B, H, N, d] raster Q, K, V (read); o_host: pinned bf16
+ * [B, H, N, d] raster O (written); lse_host: pinned fp32 [B, H, n_pad] tile-order LSE
+ * (written).  mask: n_valid = N, n_pad and block_size as the shape gives them, step inside;
+ * dense_mask: device, STATIC only.  *done (may be NULL) receives the event of `bufs` that
+ * completes once o_host and lse_host hold the results; until then the host buffers must not
+ * be touched.  Returns after enqueueing; nothing is allocated.
+ * Errors: LVA_ERR_INVALID_ARG for bad shapes, null or unpinned buffers, too few events;
+ * LVA_ERR_UNSUPPORTED for a head dim or block size without a kernel; LVA_ERR_CAPACITY when
+ * col_capacity is below lva_block_mask_max_nnz; all before anything is enqueued.  Errors of
+ * the enqueued calls are returned as they occur (work already enqueued stays enqueued).
+ */
+lva_status lva_layer_step_host(const void* qkv_host, void* o_host, float* lse_host,
+                               const lva_layer_shape* shape, const lva_mask_params* mask,
+                               const uint8_t* dense_mask, int build_mask, const int32_t* query_src,
+                               int src_heads, const lva_host_step_buffers* bufs, int head_groups,
+                               cudaStream_t compute, cudaStream_t h2d, cudaStream_t d2h,
+                               cudaEvent_t* done);
+
 /*
  * lva_device_error -- read and clear the current device's kernel error word.
  *
  * Synchronises `stream`, then stores in *status the first kernel-side fault recorded since
  * the last call (LVA_OK if none): LVA_ERR_INVALID_ARG for CSR entries out of range,
  * LVA_ERR_TIMEOUT for a pipeline wait that ran past its limit.  *detail (may be NULL)
- * receives a kernel-specific code locating the fault.
+ * receives a kernel-specific code locating the fault.  The word is taken and cleared in one
+ * atomic step on `stream`: a fault that a kernel on another stream records meanwhile is
+ * reported by this call or the next, never lost.  Concurrent calls on one device are
+ * serialised.
  */
 lva_status lva_device_error(cudaStream_t stream, lva_status* status, int* detail);
 

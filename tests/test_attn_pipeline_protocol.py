@@ -10,6 +10,9 @@ through mbarriers whose waits test a phase *parity*:
 * the softmax warps (2..9), each owning rows of S, P and O: read S_b, write P_b, rescale
   O rarely, read O in the epilogue.
 
+The LSE-only form (``lva_block_sparse_lse``) runs the same roles without the V producer,
+the P V issuer, P and O: the softmax only reads S_b and releases it.
+
 Positions T count key blocks over all the items a CTA walks, so ring slots (T mod 3), S/P
 buffers (T mod 2) and barrier phases continue from one item to the next; ``q_empty`` and
 ``o_free`` hand the single Q tile and the O accumulator from one item to the next.  Items
@@ -42,9 +45,9 @@ WARPS = 3            # softmax warps modelled (8 in the kernel; the protocol is 
 class Model(ProtocolModel):
     issuers = ("qk", "pv")
 
-    def __init__(self, items, rescale, rng, omit=()):
+    def __init__(self, items, rescale, rng, omit=(), lse_only=False):
         super().__init__(rng, omit)
-        self.items, self.rescale = items, rescale
+        self.items, self.rescale, self.lse_only = items, rescale, lse_only
         for name, count in [("q", 1), ("q_empty", 1), ("o_free", WARPS), ("final", 1), ("final_pv", 1)]:
             self.barrier(name, count)
         for s in range(KST):
@@ -65,8 +68,10 @@ class Model(ProtocolModel):
             self.buffer(f"Ow{w}")
 
     def roles(self):
-        return [self.qk_producer(), self.v_producer(), self.qk_issuer(), self.pv_issuer()] + \
-               [self.softmax(w) for w in range(WARPS)]
+        roles = [self.qk_producer(), self.qk_issuer()] + [self.softmax(w) for w in range(WARPS)]
+        if not self.lse_only:
+            roles += [self.v_producer(), self.pv_issuer()]
+        return roles
 
     # -- the roles ----------------------------------------------------------------------------
     def qk_producer(self):
@@ -151,6 +156,10 @@ class Model(ProtocolModel):
                 yield                                        # tcgen05.ld of the S rows
                 self.buf[f"S{b}w{w}"].end_read()
                 self.bar[f"s_free{b}"].arrive()
+                if self.lse_only:
+                    T += 1
+                    yield                                    # maxima, exponentials, sums
+                    continue
                 if T >= 2:
                     yield from self.wait(f"o_done{b}", (T >> 1) - 1, "p_reuse")   # P V(T-2) has read P_b
                 self.buf[f"P{b}w{w}"].begin_write(("p", T), f"sm{w}")
@@ -164,7 +173,7 @@ class Model(ProtocolModel):
                 self.bar[f"p_full{b}"].arrive()
                 T += 1
                 yield
-            if n > 0:
+            if n > 0 and not self.lse_only:
                 yield from self.wait(f"o_done{(T - 1) & 1}", (T - 1) >> 1, "epilogue")
                 self.buf[f"Ow{w}"].begin_read(("o", T - 1))
                 yield                                        # tcgen05.ld of the O rows
@@ -173,18 +182,19 @@ class Model(ProtocolModel):
             yield                                            # normalise, store O and LSE
 
 
-def _run(items, seed, omit=()):
+def _run(items, seed, omit=(), lse_only=False):
     rng = random.Random(seed)
-    Model(items, random_decisions(rng, 0.3), rng, omit).run()
+    Model(items, random_decisions(rng, 0.3), rng, omit, lse_only).run()
 
 
+@pytest.mark.parametrize("lse_only", [False, True])
 @pytest.mark.parametrize("kpc", [1, 4, 8])
-def test_random_item_runs_and_schedules(kpc):
+def test_random_item_runs_and_schedules(kpc, lse_only):
     rng = random.Random(1000 + kpc)
     for case in range(40):
         items = [rng.choice([0, 0, 1, 1, 2, 3, 5]) for _ in range(kpc)]
         for sched in range(6):
-            _run(items, seed=case * 100 + sched)
+            _run(items, seed=case * 100 + sched, lse_only=lse_only)
 
 
 @pytest.mark.parametrize("items", [
@@ -197,6 +207,7 @@ def test_random_item_runs_and_schedules(kpc):
 def test_edge_item_runs(items):
     for sched in range(30):
         _run(items, seed=sched)
+        _run(items, seed=sched, lse_only=True)
 
 
 # Each of these waits is needed on the normal path: without it (in the model only) some
@@ -205,17 +216,29 @@ WAITS = ["q_empty", "k_empty", "v_empty", "q_full", "k_full", "s_free", "p_full"
          "s_full", "p_reuse", "rescale", "epilogue"]
 
 
-@pytest.mark.parametrize("omit", WAITS)
-def test_every_wait_is_needed(omit):
+WAITS_LSE = ["q_empty", "k_empty", "q_full", "k_full", "s_free", "s_full"]
+
+
+def _caught(omit, lse_only):
     caught = 0
     for sched in range(400):
         try:
-            _run([5, 1, 3, 2], seed=sched, omit=(omit,))
+            _run([5, 1, 3, 2], seed=sched, omit=(omit,), lse_only=lse_only)
         except Hazard:
             caught += 1
             if caught >= 3:
                 break
-    assert caught > 0, f"no schedule needs the {omit} wait"
+    return caught
+
+
+@pytest.mark.parametrize("omit", WAITS)
+def test_every_wait_is_needed(omit):
+    assert _caught(omit, False) > 0, f"no schedule needs the {omit} wait"
+
+
+@pytest.mark.parametrize("omit", WAITS_LSE)
+def test_every_wait_is_needed_lse_only(omit):
+    assert _caught(omit, True) > 0, f"no schedule needs the {omit} wait (LSE only)"
 
 
 @pytest.mark.parametrize("omit", ["o_free", "final", "final_pv"])

@@ -50,6 +50,40 @@ int main(void) {
   printf("attn null %s: %s\n", lva_status_string(s), lva_last_error_message());
   s = lva_selftest_wait(7, (cudaStream_t)0);
   printf("selftest %s\n", lva_status_string(s));
+  {
+    /* the host-buffer layer step: every argument check runs before any stream or device work */
+    lva_layer_shape sh;
+    lva_host_step_buffers hb;
+    cudaEvent_t ev[16];
+    char host[64];
+    memset(&sh, 0, sizeof(sh));
+    memset(&hb, 0, sizeof(hb));
+    memset(ev, 0, sizeof(ev));
+    sh.B = 1; sh.H = 12; sh.d = 128; sh.block_size = 128; sh.T = 21; sh.Hg = 30; sh.Wg = 52;
+    sh.tile_t = 1; sh.tile_h = 8; sh.tile_w = 16; sh.scale = 0.088388f;
+    p.block_size = 128;
+    s = lva_layer_step_host(host, host, (float*)host, NULL, &p, NULL, 1, NULL, 1, &hb, 6, 0, 0, 0, NULL);
+    printf("step null %s: %s\n", lva_status_string(s), lva_last_error_message());
+    sh.d = 96;
+    s = lva_layer_step_host(host, host, (float*)host, &sh, &p, NULL, 1, NULL, 1, &hb, 6, 0, 0, 0, NULL);
+    printf("step d96 %s\n", lva_status_string(s));
+    sh.d = 128;
+    s = lva_layer_step_host(host, host, (float*)host, &sh, &p, NULL, 1, NULL, 1, &hb, 6, 0, 0, 0, NULL);
+    printf("step buffers %s: %s\n", lva_status_string(s), lva_last_error_message());
+    hb.qkv_stage = hb.o_stage = hb.qkv_tile = (void*)(uintptr_t)256;
+    hb.lse_stage = (float*)(uintptr_t)256;
+    hb.row_ptr = hb.col_idx = hb.nnz = (int32_t*)(uintptr_t)256;
+    hb.events = ev;
+    hb.num_events = 16;
+    hb.col_capacity = cap - 1;
+    hb.col_len = cap - 1;
+    s = lva_layer_step_host(host, host, (float*)host, &sh, &p, NULL, 1, NULL, 1, &hb, 6, 0, 0, 0, NULL);
+    printf("step capacity %s\n", lva_status_string(s));
+    hb.col_capacity = cap;
+    hb.num_events = 2 * 6 + 1;
+    s = lva_layer_step_host(host, host, (float*)host, &sh, &p, NULL, 1, NULL, 1, &hb, 6, 0, 0, 0, NULL);
+    printf("step events %s: %s\n", lva_status_string(s), lva_last_error_message());
+  }
   return 0;
 }
 """
@@ -82,3 +116,9 @@ def test_c_program_calls_the_library(program):
     assert out[5] == "attn LVA_ERR_UNSUPPORTED"          # head dim 96
     assert out[6] == "attn null LVA_ERR_INVALID_ARG: attn: null pointer"
     assert out[7] == "selftest LVA_ERR_INVALID_ARG"      # unknown mode
+    assert out[8] == "step null LVA_ERR_INVALID_ARG: layer_step_host: null shape, mask or buffers"
+    assert out[9] == "step d96 LVA_ERR_UNSUPPORTED"
+    assert out[10] == "step buffers LVA_ERR_INVALID_ARG: layer_step_host: null device buffer or event array"
+    assert out[11] == "step capacity LVA_ERR_CAPACITY"       # col_capacity below the mask's maximum
+    assert out[12] == ("step events LVA_ERR_INVALID_ARG: layer_step_host: too few events "
+                       "(need 2 * groups + 2)")       # 6 groups of 2 heads need 14 events

@@ -142,6 +142,61 @@ def test_corrupt_csr_is_reported_not_faulted():
     assert status == 1 and detail == 3
 
 
+def test_repeated_column_is_reported_not_counted_twice():
+    """A CSR row that lists a key block twice (not strictly ascending) is skipped and
+    reported, never attended twice."""
+    import block_sparse_attention_lva_b200 as lva
+    dev = require_gpu()
+    B, H, n_pad, d, bs = 1, 1, 512, 128, 128
+    q, k, v = (_rand_bf16((B, H, n_pad, d), s) for s in (11, 12, 13))
+    row_ptr = torch.tensor([0, 2, 4, 6, 8], dtype=torch.int32, device=dev)
+    col_idx = torch.tensor([0, 1, 2, 2, 1, 3, 0, 3], dtype=torch.int32, device=dev)   # row 1 repeats 2
+    o = torch.empty((B, H, n_pad, d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, H, n_pad), dtype=torch.float32, device=dev)
+    lva.lva_block_sparse_attn(q.to(dev), k.to(dev), v.to(dev), o, lse, n_pad, bs, row_ptr, col_idx, 1, 0.1)
+    status, detail = lva.lva_device_error()
+    assert status == 1 and detail == 1
+    assert torch.all(o[0, 0, 128:256] == 0) and torch.all(torch.isneginf(lse[0, 0, 128:256]))
+    m = np.zeros((1, 4, 4), bool)
+    m[0, 0, [0, 1]] = True
+    m[0, 2, [1, 3]] = True
+    m[0, 3, [0, 3]] = True
+    o_ref, lse_ref = attention_blocked(q, k, v, m, bs, n_pad, 0.1)
+    keep = np.r_[0:128, 256:512]
+    check_o_lse(o[:, :, keep], lse[:, :, keep], o_ref[:, :, keep], lse_ref[:, :, keep], "repeated column")
+
+
+@pytest.mark.parametrize("B,H,n_pad,n_valid,d,bs,hm,density,seed", [
+    (1, 3, 2048, 2000, 128, 128, 3, 0.5, 21),
+    (2, 2, 1024, 1024, 64, 128, 1, 1.0, 22),
+    (1, 2, 768, 700, 128, 64, 2, 0.4, 23),
+])
+def test_lse_only_matches_attention_lse(B, H, n_pad, n_valid, d, bs, hm, density, seed):
+    """lva_block_sparse_lse gives the LSE of lva_block_sparse_attn (same scores, maxima and
+    sums) and matches the oracle; empty rows give -inf."""
+    import block_sparse_attention_lva_b200 as lva
+    dev = require_gpu()
+    q, k, v = (_rand_bf16((B, H, n_pad, d), seed + 100 * t) for t in range(3))
+    nb = n_pad // bs
+    masks = np.random.default_rng(seed).random((hm, nb, nb)) < density
+    masks[0, 1] = False                                      # an empty row
+    scale = 1.0 / math.sqrt(d)
+    _, lse_full = _attn_gpu(q, k, v, masks, bs, n_valid, scale)
+    rp, ci = dense_to_csr(masks)
+    lse = torch.full((B, H, n_pad), float("nan"), dtype=torch.float32, device=dev)
+    lva.lva_block_sparse_lse(q.to(dev), k.to(dev), lse, n_valid, bs, torch.from_numpy(rp).to(dev),
+                             torch.from_numpy(ci).to(dev), hm, scale)
+    torch.cuda.synchronize()
+    assert lva.lva_device_error() == (0, 0)
+    a, b = lse.cpu().numpy(), lse_full.cpu().numpy()
+    assert np.array_equal(np.isneginf(a), np.isneginf(b))
+    fin = np.isfinite(b)
+    assert np.abs(a[fin] - b[fin]).max() <= 1e-5
+    _, lse_ref = attention_blocked(q, k, v, masks, bs, n_valid, scale)
+    assert np.array_equal(np.isneginf(a), np.isneginf(lse_ref))
+    assert np.abs(a[fin] - lse_ref[fin]).max() <= 1e-3
+
+
 # ---------------------------------------------------------------- full workloads
 def _oracle_mask(w, spec, step):
     if spec["kind"] == "window_anchor":
