@@ -587,21 +587,28 @@ def run_report(args):
                           "kernel_error": status}), flush=True)
         del qd, kd, cal, samples, out, mask
         torch.cuda.empty_cache()
-    # mask-builder stress size: static mask, 40 heads x 4096 x 4096 blocks (671 MB read)
+    # mask-builder stress size: static mask, 40 heads x 4096 x 4096 blocks (671 MB read), or
+    # --stress-heads heads of 4096 x 4096 blocks
     if "stress" in names or args.report_stress:
-        hm, nb = 40, 4096
+        hm, nb = args.stress_heads, 4096
         g = torch.Generator(device=dev).manual_seed(5)
         dense = (torch.rand((hm, nb, nb), generator=g, device=dev) < 0.3).to(torch.uint8)
         params = lva.MaskParams(lva.LVA_MASK_STATIC, nb * 128, nb * 128, 128, hm)
         row_ptr = torch.empty(hm * nb + 1, dtype=torch.int32, device=dev)
         col_idx = torch.empty(lva.lva_block_mask_max_nnz(params), dtype=torch.int32, device=dev)
         nnz = torch.empty(1, dtype=torch.int32, device=dev)
-        ms = _time_cuda(lambda: lva.lva_build_block_mask(params, dense, row_ptr, col_idx, nnz))
+        ws = torch.empty(lva.lva_block_mask_workspace_bytes(params), dtype=torch.uint8, device=dev)
+        ms_two_read = _time_cuda(lambda: lva.lva_build_block_mask(params, dense, row_ptr, col_idx, nnz))
+        ms = _time_cuda(lambda: lva.lva_build_block_mask_ws(params, dense, row_ptr, col_idx, nnz, ws))
         n = int(nnz.item())
+        # algorithmic bytes: the dense mask read once, row_ptr and col_idx written once
         byts = hm * nb * nb + 4 * (hm * nb + 1) + 4 * n
-        print(json.dumps({"report": "mask_stress", "mask_heads": hm, "nb": nb, "nnz": n, "ms": ms,
-                          "gbs": byts / ms / 1e6, "hbm_peak_gbs": hbm}), flush=True)
-        del dense, col_idx
+        print(json.dumps({"report": "mask_stress", "mask_heads": hm, "nb": nb, "nnz": n,
+                          "ms_workspace_build": ms, "gbs": byts / ms / 1e6, "frac_of_hbm": byts / ms / 1e6 / hbm,
+                          "ms_two_read_build": ms_two_read, "gbs_two_read": byts / ms_two_read / 1e6,
+                          "algorithmic_bytes": byts, "workspace_bytes": ws.numel(), "hbm_peak_gbs": hbm}),
+              flush=True)
+        del dense, col_idx, ws
         torch.cuda.empty_cache()
     if "oracle" in names:
         run_oracle_report(args, gpu_ms)
@@ -619,6 +626,7 @@ def main():
     ap.add_argument("--report", default="", help="comma list of workloads (tiny,small,static,large,long,stress,squad,calib,oracle): "
                     "per-mask kernel timings and the density sweep fit instead of the bench line")
     ap.add_argument("--report-stress", action="store_true")
+    ap.add_argument("--stress-heads", type=int, default=40, help="mask heads of the 4096 x 4096-block stress build")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

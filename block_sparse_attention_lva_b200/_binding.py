@@ -60,6 +60,9 @@ SIGNATURES = {
                                     _c_i64, _c_i64, _c_int, _c_int, _vp]),
     "lva_block_mask_max_nnz": (_c_i64, [ctypes.POINTER(LvaMaskParams)]),
     "lva_build_block_mask": (_c_int, [ctypes.POINTER(LvaMaskParams), _vp, _vp, _vp, _c_i64, _vp, _vp]),
+    "lva_block_mask_workspace_bytes": (_c_i64, [ctypes.POINTER(LvaMaskParams)]),
+    "lva_build_block_mask_ws": (_c_int, [ctypes.POINTER(LvaMaskParams), _vp, _vp, _vp, _c_i64, _vp, _vp, _c_i64,
+                                         _vp]),
     "lva_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
                                        _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp, _c_int, _vp]),
     "lva_block_sparse_lse": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int, _c_int, _vp, _vp,
@@ -201,6 +204,34 @@ def lva_build_block_mask(params: MaskParams, dense_mask, row_ptr, col_idx, nnz_o
     _check(lib.lva_build_block_mask(ctypes.byref(cp), _ptr(dense_mask), _ptr(row_ptr), _ptr(col_idx),
                                     col_idx.numel(), _ptr(nnz_out),
                                     ctypes.c_void_p(_stream(row_ptr.device))))
+    return row_ptr, col_idx, nnz_out
+
+
+def lva_block_mask_workspace_bytes(params: MaskParams) -> int:
+    cp = params.to_c()
+    return lib.lva_block_mask_workspace_bytes(ctypes.byref(cp))
+
+
+def lva_build_block_mask_ws(params: MaskParams, dense_mask, row_ptr, col_idx, nnz_out, workspace):
+    """``lva_build_block_mask`` with a caller-owned device workspace (uint8 tensor of at least
+    ``lva_block_mask_workspace_bytes(params)`` bytes; may be None when that is 0)."""
+    import torch
+    nb = params.n_pad // params.block_size
+    _cuda_tensor(row_ptr, "row_ptr", torch.int32, params.mask_heads * nb + 1)
+    _cuda_tensor(col_idx, "col_idx", torch.int32)
+    _cuda_tensor(nnz_out, "nnz_out", torch.int32, 1)
+    if params.kind == LVA_MASK_STATIC:
+        _cuda_tensor(dense_mask, "dense_mask", torch.uint8, params.mask_heads * nb * nb)
+    else:
+        dense_mask = None
+    ws_bytes = 0
+    if workspace is not None:
+        _cuda_tensor(workspace, "workspace")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    cp = params.to_c()
+    _check(lib.lva_build_block_mask_ws(ctypes.byref(cp), _ptr(dense_mask), _ptr(row_ptr), _ptr(col_idx),
+                                       col_idx.numel(), _ptr(nnz_out), _ptr(workspace), ws_bytes,
+                                       ctypes.c_void_p(_stream(row_ptr.device))))
     return row_ptr, col_idx, nnz_out
 
 

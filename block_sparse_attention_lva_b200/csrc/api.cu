@@ -170,9 +170,9 @@ int64_t lva_block_mask_max_nnz(const lva_mask_params* p) {
   return int64_t(p->mask_heads) * nb * nb;
 }
 
-lva_status lva_build_block_mask(const lva_mask_params* p, const uint8_t* dense_mask, int32_t* row_ptr,
-                                int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
-                                cudaStream_t stream) {
+// Checks shared by both mask-build calls; fills the launcher arguments.
+static lva_status mask_args(const lva_mask_params* p, const uint8_t* dense_mask, int32_t* row_ptr,
+                            int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out, MaskArgs* a) {
   lva_status s = check_mask_params(p);
   if (s != LVA_OK) return s;
   if (row_ptr == nullptr || col_idx == nullptr || nnz_out == nullptr)
@@ -184,23 +184,52 @@ lva_status lva_build_block_mask(const lva_mask_params* p, const uint8_t* dense_m
   const int64_t need = lva_block_mask_max_nnz(p);
   if (col_capacity < need)
     return fail(LVA_ERR_CAPACITY, "mask: col_capacity %lld < %lld", (long long)col_capacity, (long long)need);
+  a->kind = p->kind;
+  a->mask_heads = p->mask_heads;
+  a->block_size = p->block_size;
+  a->n_pad = p->n_pad;
+  a->n_valid = p->n_valid;
+  a->unit_tokens = p->window_unit_tokens;
+  a->radius = p->window_radius;
+  a->num_anchors = p->num_anchors;
+  a->step = p->step;
+  a->group_blocks = p->group_blocks;
+  a->budget_frames = p->budget_frames;
+  a->dense = dense_mask;
+  a->row_ptr = row_ptr;
+  a->col_idx = col_idx;
+  a->nnz_out = nnz_out;
+  return LVA_OK;
+}
+
+lva_status lva_build_block_mask(const lva_mask_params* p, const uint8_t* dense_mask, int32_t* row_ptr,
+                                int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
+                                cudaStream_t stream) {
   MaskArgs a;
-  a.kind = p->kind;
-  a.mask_heads = p->mask_heads;
-  a.block_size = p->block_size;
-  a.n_pad = p->n_pad;
-  a.n_valid = p->n_valid;
-  a.unit_tokens = p->window_unit_tokens;
-  a.radius = p->window_radius;
-  a.num_anchors = p->num_anchors;
-  a.step = p->step;
-  a.group_blocks = p->group_blocks;
-  a.budget_frames = p->budget_frames;
-  a.dense = dense_mask;
-  a.row_ptr = row_ptr;
-  a.col_idx = col_idx;
-  a.nnz_out = nnz_out;
+  const lva_status s = mask_args(p, dense_mask, row_ptr, col_idx, col_capacity, nnz_out, &a);
+  if (s != LVA_OK) return s;
   return from_cuda(launch_build_mask(a, stream), "mask launch");
+}
+
+int64_t lva_block_mask_workspace_bytes(const lva_mask_params* p) {
+  if (check_mask_params(p) != LVA_OK) return -1;
+  const int64_t nb = p->n_pad / p->block_size;
+  return mask_workspace_bytes(p->kind, int64_t(p->mask_heads) * nb, nb);
+}
+
+lva_status lva_build_block_mask_ws(const lva_mask_params* p, const uint8_t* dense_mask, int32_t* row_ptr,
+                                   int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out, void* workspace,
+                                   int64_t workspace_bytes, cudaStream_t stream) {
+  MaskArgs a;
+  const lva_status s = mask_args(p, dense_mask, row_ptr, col_idx, col_capacity, nnz_out, &a);
+  if (s != LVA_OK) return s;
+  const int64_t need = lva_block_mask_workspace_bytes(p);
+  if (need == 0) return from_cuda(launch_build_mask(a, stream), "mask launch");
+  if (workspace == nullptr) return fail(LVA_ERR_INVALID_ARG, "mask: null workspace");
+  if (!aligned(workspace, 16)) return fail(LVA_ERR_INVALID_ARG, "mask: workspace must be 16-byte aligned");
+  if (workspace_bytes < need)
+    return fail(LVA_ERR_CAPACITY, "mask: workspace_bytes %lld < %lld", (long long)workspace_bytes, (long long)need);
+  return from_cuda(launch_build_mask_packed(a, workspace, stream), "mask launch");
 }
 
 static lva_status attn_common(const char* fn, const void* q, const void* k, const void* v, void* o,

@@ -102,21 +102,6 @@ __global__ void aggregate_kernel(const uint8_t* __restrict__ masks, uint8_t* __r
   }
 }
 
-int sm_count() {
-  static std::atomic<int> cached[kMaxCachedDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  const bool cacheable = dev >= 0 && dev < kMaxCachedDevices;
-  if (cacheable) {
-    const int c = cached[dev].load(std::memory_order_relaxed);
-    if (c > 0) return c;
-  }
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-  if (cacheable) cached[dev].store(n, std::memory_order_relaxed);
-  return n;
-}
-
 }  // namespace
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {

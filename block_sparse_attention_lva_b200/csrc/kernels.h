@@ -31,6 +31,23 @@ cudaError_t once_per_device(DeviceFlags& done, F&& setup) {
   return e;
 }
 
+// Streaming multiprocessors of the current device (looked up once per device; 148 if the
+// query fails).
+inline int sm_count() {
+  static std::atomic<int> cached[kMaxCachedDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const bool cacheable = dev >= 0 && dev < kMaxCachedDevices;
+  if (cacheable) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (cacheable) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 struct ReorderArgs {
   const void* src;
   void* dst;
@@ -55,6 +72,12 @@ struct MaskArgs {
   int32_t* nnz_out;
 };
 cudaError_t launch_build_mask(const MaskArgs& a, cudaStream_t stream);
+
+// Workspace bytes of the packed static-mask build (0 for the other kinds), and the build
+// itself: the dense mask is read once into bits (workspace), the counts are scanned by
+// several CTAs when there are many rows, and the bits are expanded into the CSR.
+int64_t mask_workspace_bytes(int kind, int64_t rows, int64_t nb);
+cudaError_t launch_build_mask_packed(const MaskArgs& a, void* workspace, cudaStream_t stream);
 
 struct AttnArgs {
   const void* q;

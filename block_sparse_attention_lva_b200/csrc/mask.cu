@@ -186,15 +186,15 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32) mask_rows_kernel(MaskDev 
 constexpr int kScanThreads = 1024;
 constexpr int kScanPer = 4;  // elements per thread per tile
 
-// In-place inclusive scan of row_ptr[1..R] by a single CTA, tile by tile; nnz = total.
-__global__ void __launch_bounds__(kScanThreads) mask_scan_kernel(int32_t* row_ptr, int64_t R,
-                                                                 int32_t* nnz_out) {
+// In-place inclusive scan of a[0..R) by a single CTA, tile by tile; *total_out = the sum
+// (for the CSR: a = row_ptr + 1, total = nnz).
+__global__ void __launch_bounds__(kScanThreads) mask_scan_kernel(int32_t* a, int64_t R,
+                                                                 int32_t* total_out) {
   __shared__ int32_t warp_sums[kScanThreads / 32];
   __shared__ int32_t carry_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) carry_s = 0;
   __syncthreads();
-  int32_t* a = row_ptr + 1;
   for (int64_t t0 = 0; t0 < R; t0 += int64_t(kScanThreads) * kScanPer) {
     int32_t v[kScanPer];
     int32_t local = 0;
@@ -234,10 +234,200 @@ __global__ void __launch_bounds__(kScanThreads) mask_scan_kernel(int32_t* row_pt
     if (tid == kScanThreads - 1) carry_s = carry + warp_sums[31];
     __syncthreads();
   }
-  if (tid == 0) *nnz_out = carry_s;
+  if (tid == 0) *total_out = carry_s;
+}
+
+constexpr int kScanTile = kScanThreads * kScanPer;   // elements per CTA of the tiled scan
+
+// Tiled scan: every CTA scans its tile of a[0..R) in place (inclusive, local) and
+// writes the tile's sum to sums[tile].
+__global__ void __launch_bounds__(kScanThreads) scan_tiles_kernel(int32_t* a, int64_t R, int32_t* sums) {
+  __shared__ int32_t warp_sums[kScanThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t0 = int64_t(blockIdx.x) * kScanTile;
+  int32_t v[kScanPer];
+  int32_t local = 0;
+#pragma unroll
+  for (int e = 0; e < kScanPer; ++e) {
+    const int64_t idx = t0 + int64_t(tid) * kScanPer + e;
+    v[e] = idx < R ? a[idx] : 0;
+    local += v[e];
+  }
+  int32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t ws = warp_sums[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t t = __shfl_up_sync(0xffffffffu, ws, o);
+      if (lane >= o) ws += t;
+    }
+    warp_sums[lane] = ws;
+  }
+  __syncthreads();
+  int32_t run = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - local;
+#pragma unroll
+  for (int e = 0; e < kScanPer; ++e) {
+    const int64_t idx = t0 + int64_t(tid) * kScanPer + e;
+    run += v[e];
+    if (idx < R) a[idx] = run;
+  }
+  if (tid == kScanThreads - 1) sums[blockIdx.x] = warp_sums[31];
+}
+
+// The 16 nonzero-byte flags of a 16-byte vector as 16 bits (bit b = byte b is nonzero).
+__device__ __forceinline__ uint32_t nonzero_bits16(uint4 v) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  uint32_t m = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t t = ((((w[k] & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w[k]) & 0x80808080u) >> 7;   // bits 0, 8, 16, 24
+    t = (t | (t >> 7) | (t >> 14) | (t >> 21)) & 0xFu;
+    m |= t << (4 * k);
+  }
+  return m;
+}
+
+constexpr int kPackWarps = 8;
+
+// Static masks, pass 1: one warp per row reads the dense row once (16 bytes per lane) and
+// writes it as bits -- bit j of word j / 32 of the packed row (wpr words, the tail words
+// zero) -- and its count to cnt[row].
+__global__ void __launch_bounds__(kPackWarps * 32) mask_pack_kernel(const uint8_t* dense, int64_t rows, int64_t nb,
+                                                                  int64_t wpr, uint32_t* packed, int32_t* cnt) {
+  const int lane = threadIdx.x & 31;
+  for (int64_t row = int64_t(blockIdx.x) * kPackWarps + (threadIdx.x >> 5); row < rows;
+       row += int64_t(gridDim.x) * kPackWarps) {
+    const uint8_t* src = dense + row * nb;
+    uint32_t* dst = packed + row * wpr;
+    int32_t count = 0;
+    if (nb % 16 == 0 && (reinterpret_cast<uintptr_t>(dense) & 15) == 0) {
+      // up to 4096 columns per round: all of a lane's loads are issued before any is used
+      constexpr int kLoads = 8;
+      for (int64_t r0 = 0; r0 < nb; r0 += 512 * kLoads) {
+        uint4 v[kLoads];
+#pragma unroll
+        for (int u = 0; u < kLoads; ++u) {
+          const int64_t j = r0 + u * 512 + lane * 16;
+          v[u] = j < nb ? __ldcs(reinterpret_cast<const uint4*>(src + j)) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kLoads; ++u) {
+          const int64_t j0 = r0 + u * 512, j = j0 + lane * 16;
+          const uint32_t m16 = nonzero_bits16(v[u]);
+          count += __popc(m16);
+          const uint32_t hi = __shfl_down_sync(0xffffffffu, m16, 1);
+          if (!(lane & 1) && j < nb) dst[j0 / 32 + lane / 2] = m16 | (hi << 16);
+        }
+      }
+      count = __reduce_add_sync(0xffffffffu, count);
+    } else {
+      for (int64_t j0 = 0; j0 < nb; j0 += 32) {
+        const int64_t j = j0 + lane;
+        const uint32_t b = __ballot_sync(0xffffffffu, j < nb && src[j] != 0);
+        if (lane == 0) dst[j0 / 32] = b;
+        count += __popc(b);
+      }
+    }
+    for (int64_t w = (nb + 31) / 32 + lane; w < wpr; w += 32) dst[w] = 0;
+    if (lane == 0) cnt[row] = count;
+  }
+}
+
+// Static masks, pass 3: one warp per row.  Its CSR offsets come from the tile-local
+// inclusive scan of the counts (cnt) plus the scanned tile sums (sums, absent for a single
+// tile); the warp writes row_ptr[row + 1] and expands the packed bits into ascending column
+// indices, 1024 columns (one word per lane) at a time: each lane writes its set bits into a
+// shared-memory staging run at its exclusive prefix count, then the warp copies the run to
+// col_idx with coalesced stores.  The next round's words are loaded before this round is
+// expanded.
+__global__ void __launch_bounds__(kPackWarps * 32) mask_fill_packed_kernel(const uint32_t* packed, int64_t rows,
+                                                                         int64_t nb, int64_t wpr,
+                                                                         const int32_t* cnt, const int32_t* sums,
+                                                                         int32_t* row_ptr, int32_t* col_idx) {
+  __shared__ int32_t stage[kPackWarps][1024];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t* st = stage[warp];
+  for (int64_t row = int64_t(blockIdx.x) * kPackWarps + warp; row < rows; row += int64_t(gridDim.x) * kPackWarps) {
+    const int64_t tile = row / kScanTile;
+    const int32_t off = (sums != nullptr && tile > 0) ? sums[tile - 1] : 0;
+    int32_t base = off + ((row % kScanTile) > 0 ? cnt[row - 1] : 0);
+    if (lane == 0) {
+      row_ptr[row + 1] = off + cnt[row];
+      if (row == 0) row_ptr[0] = 0;
+    }
+    const uint32_t* src = packed + row * wpr;
+    const int64_t nw = (nb + 31) / 32;
+    uint32_t next = lane < nw ? __ldcs(src + lane) : 0u;
+    for (int64_t w0 = 0; w0 < nw; w0 += 32) {
+      uint32_t word = next;
+      next = w0 + 32 + lane < nw ? __ldcs(src + w0 + 32 + lane) : 0u;
+      const int c = __popc(word);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      int pos = incl - c;
+      const int32_t col0 = int32_t((w0 + lane) * 32);
+      while (word != 0u) {
+        st[pos++] = col0 + (__ffs(word) - 1);
+        word &= word - 1u;
+      }
+      __syncwarp();
+      for (int k = lane; k < total; k += 32) col_idx[base + k] = st[k];
+      __syncwarp();
+      base += total;
+    }
+  }
 }
 
 }  // namespace
+
+// Workspace: the packed rows (rows x wpr words), the row counts (rows words, scanned in
+// place tile by tile) and the tile sums.
+int64_t mask_workspace_bytes(int kind, int64_t rows, int64_t nb) {
+  if (kind != kStatic) return 0;
+  const int64_t wpr = ((nb + 31) / 32 + 3) / 4 * 4;
+  const int64_t tiles = (rows + kScanTile - 1) / kScanTile;
+  return rows * wpr * 4 + (rows * 4 + 15) / 16 * 16 + (tiles * 4 + 15) / 16 * 16;
+}
+
+cudaError_t launch_build_mask_packed(const MaskArgs& a, void* workspace, cudaStream_t stream) {
+  const int64_t nb = a.n_pad / a.block_size;
+  const int64_t rows = int64_t(a.mask_heads) * nb;
+  const int64_t wpr = ((nb + 31) / 32 + 3) / 4 * 4;
+  uint32_t* packed = static_cast<uint32_t*>(workspace);
+  int32_t* cnt = reinterpret_cast<int32_t*>(packed + rows * wpr);
+  int32_t* sums = cnt + (rows + 3) / 4 * 4;
+  const int64_t tiles = (rows + kScanTile - 1) / kScanTile;
+  // One warp per row (a grid-stride form with one wave of CTAs measured slower).
+  const unsigned pack_blocks = unsigned((rows + kPackWarps - 1) / kPackWarps);
+  const unsigned fill_blocks = pack_blocks;
+  mask_pack_kernel<<<pack_blocks, kPackWarps * 32, 0, stream>>>(a.dense, rows, nb, wpr, packed, cnt);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (tiles == 1) {
+    mask_scan_kernel<<<1, kScanThreads, 0, stream>>>(cnt, rows, a.nnz_out);
+  } else {
+    scan_tiles_kernel<<<unsigned(tiles), kScanThreads, 0, stream>>>(cnt, rows, sums);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mask_scan_kernel<<<1, kScanThreads, 0, stream>>>(sums, tiles, a.nnz_out);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  mask_fill_packed_kernel<<<fill_blocks, kPackWarps * 32, 0, stream>>>(packed, rows, nb, wpr, cnt,
+                                                                  tiles == 1 ? nullptr : sums, a.row_ptr,
+                                                                  a.col_idx);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_build_mask(const MaskArgs& a, cudaStream_t stream) {
   MaskDev m;
@@ -258,7 +448,7 @@ cudaError_t launch_build_mask(const MaskArgs& a, cudaStream_t stream) {
   mask_rows_kernel<false><<<blocks, kWarpsPerBlock * 32, 0, stream>>>(m, a.row_ptr, a.col_idx);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  mask_scan_kernel<<<1, kScanThreads, 0, stream>>>(a.row_ptr, m.rows, a.nnz_out);
+  mask_scan_kernel<<<1, kScanThreads, 0, stream>>>(a.row_ptr + 1, m.rows, a.nnz_out);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   mask_rows_kernel<true><<<blocks, kWarpsPerBlock * 32, 0, stream>>>(m, a.row_ptr, a.col_idx);

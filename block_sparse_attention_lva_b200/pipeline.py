@@ -86,6 +86,9 @@ class VideoBlockSparseAttention:
         self.row_ptr = torch.empty(self.mask_heads * self.nb + 1, dtype=torch.int32, **kw)
         self.col_idx = torch.empty(cap, dtype=torch.int32, **kw)
         self.nnz = torch.empty(1, dtype=torch.int32, **kw)
+        # Static masks are built through the workspace path (the dense mask read once).
+        ws = lb.lva_block_mask_workspace_bytes(self.params)
+        self.mask_ws = torch.empty(ws, dtype=torch.uint8, **kw) if ws > 0 else None
         self.query_src = (torch.as_tensor(query_src, dtype=torch.int32).to(self.device).contiguous()
                           if query_src is not None else None)
         if self.query_src is not None and (self.query_src.dim() != 2 or self.query_src.shape[0] not in (1, H)
@@ -101,7 +104,8 @@ class VideoBlockSparseAttention:
         if self._built_step == key:
             return
         self.params.step = key
-        lb.lva_build_block_mask(self.params, self.dense_mask, self.row_ptr, self.col_idx, self.nnz)
+        lb.lva_build_block_mask_ws(self.params, self.dense_mask, self.row_ptr, self.col_idx, self.nnz,
+                                   self.mask_ws)
         self._built_step = key
         # A mask built once can tell the attention call its exact entry count (read back once);
         # short rows then get CTAs that walk several query blocks.  Per-step masks keep the

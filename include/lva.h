@@ -154,6 +154,38 @@ lva_status lva_build_block_mask(const lva_mask_params* params, const uint8_t* de
                                 int32_t* nnz_out, cudaStream_t stream);
 
 /*
+ * lva_block_mask_workspace_bytes -- device workspace of lva_build_block_mask_ws.
+ *
+ * Bytes of the caller-owned workspace that lva_build_block_mask_ws needs for these
+ * parameters: for STATIC, one bit per block pair (mask_heads * nb rows of
+ * ceil(nb / 128) * 16 bytes), 4 bytes per row and 4 bytes per 4096 rows (each rounded up to
+ * 16 bytes); 0 for the parametric kinds.
+ * Returns -1 for invalid parameters.
+ */
+int64_t lva_block_mask_workspace_bytes(const lva_mask_params* params);
+
+/*
+ * lva_build_block_mask_ws -- lva_build_block_mask with a caller-owned device workspace.
+ *
+ * The same CSR, bit for bit, as lva_build_block_mask.  For STATIC masks the dense input is
+ * read once: a first pass writes every row as bits (into `workspace`) and its count, the
+ * counts are scanned (by several CTAs when there are more than 4096 rows), and a last pass
+ * expands the bits into the column lists.  lva_build_block_mask reads the dense mask twice
+ * instead (a count pass and a fill pass) and needs no workspace.  The parametric kinds need
+ * none here either (workspace may then be NULL).
+ *
+ * workspace: device, 16-byte aligned, at least lva_block_mask_workspace_bytes(params)
+ * bytes (its contents are overwritten; it may be reused once the call has completed on
+ * `stream`).  Other arguments and errors as for lva_build_block_mask; in addition
+ * LVA_ERR_INVALID_ARG for a null or misaligned workspace and LVA_ERR_CAPACITY when
+ * workspace_bytes is too small.
+ */
+lva_status lva_build_block_mask_ws(const lva_mask_params* params, const uint8_t* dense_mask,
+                                   int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                   int32_t* nnz_out, void* workspace, int64_t workspace_bytes,
+                                   cudaStream_t stream);
+
+/*
  * lva_block_sparse_attn -- softmax attention computed only on listed block pairs.
  *
  * The block-sparse attention of the LVSA page (technical summary section 2: attention
