@@ -63,6 +63,7 @@ SIGNATURES = {
     "lva_block_mask_workspace_bytes": (_c_i64, [ctypes.POINTER(LvaMaskParams)]),
     "lva_build_block_mask_ws": (_c_int, [ctypes.POINTER(LvaMaskParams), _vp, _vp, _vp, _c_i64, _vp, _vp, _c_i64,
                                          _vp]),
+    "lva_build_block_mask_noalloc": (_c_int, [ctypes.POINTER(LvaMaskParams), _vp, _vp, _vp, _c_i64, _vp, _vp]),
     "lva_block_sparse_attn": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int,
                                        _c_int, _vp, _vp, _c_i64, _c_int, ctypes.c_float, _vp, _c_int, _vp]),
     "lva_block_sparse_lse": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _c_i64, _c_i64, _c_int, _c_int, _vp, _vp,
@@ -232,6 +233,24 @@ def lva_build_block_mask_ws(params: MaskParams, dense_mask, row_ptr, col_idx, nn
     _check(lib.lva_build_block_mask_ws(ctypes.byref(cp), _ptr(dense_mask), _ptr(row_ptr), _ptr(col_idx),
                                        col_idx.numel(), _ptr(nnz_out), _ptr(workspace), ws_bytes,
                                        ctypes.c_void_p(_stream(row_ptr.device))))
+    return row_ptr, col_idx, nnz_out
+
+
+def lva_build_block_mask_noalloc(params: MaskParams, dense_mask, row_ptr, col_idx, nnz_out):
+    """``lva_build_block_mask_ws`` with the scratch in the library's own 16 MiB device array
+    (no workspace argument; nothing is allocated by the call)."""
+    import torch
+    nb = params.n_pad // params.block_size
+    _cuda_tensor(row_ptr, "row_ptr", torch.int32, params.mask_heads * nb + 1)
+    _cuda_tensor(col_idx, "col_idx", torch.int32)
+    _cuda_tensor(nnz_out, "nnz_out", torch.int32, 1)
+    if params.kind == LVA_MASK_STATIC:
+        _cuda_tensor(dense_mask, "dense_mask", torch.uint8, params.mask_heads * nb * nb)
+    else:
+        dense_mask = None
+    cp = params.to_c()
+    _check(lib.lva_build_block_mask_noalloc(ctypes.byref(cp), _ptr(dense_mask), _ptr(row_ptr), _ptr(col_idx),
+                                            col_idx.numel(), _ptr(nnz_out), ctypes.c_void_p(_stream(row_ptr.device))))
     return row_ptr, col_idx, nnz_out
 
 

@@ -232,6 +232,21 @@ lva_status lva_build_block_mask_ws(const lva_mask_params* p, const uint8_t* dens
   return from_cuda(launch_build_mask_packed(a, workspace, stream), "mask launch");
 }
 
+lva_status lva_build_block_mask_noalloc(const lva_mask_params* p, const uint8_t* dense_mask, int32_t* row_ptr,
+                                        int32_t* col_idx, int64_t col_capacity, int32_t* nnz_out,
+                                        cudaStream_t stream) {
+  MaskArgs a;
+  const lva_status s = mask_args(p, dense_mask, row_ptr, col_idx, col_capacity, nnz_out, &a);
+  if (s != LVA_OK) return s;
+  const int64_t need = lva_block_mask_workspace_bytes(p);
+  if (need > mask_noalloc_scratch_bytes())
+    return fail(LVA_ERR_CAPACITY,
+                "mask_noalloc: these parameters need %lld bytes of scratch; the library holds %lld "
+                "(use lva_build_block_mask_ws with a workspace, or lva_build_block_mask)",
+                (long long)need, (long long)mask_noalloc_scratch_bytes());
+  return from_cuda(launch_build_mask_noalloc(a, stream), "mask_noalloc launch");
+}
+
 static lva_status attn_common(const char* fn, const void* q, const void* k, const void* v, void* o,
                               float* lse, int B, int H, int64_t n_pad, int64_t n_valid, int d,
                               int block_size, const int32_t* row_ptr, const int32_t* col_idx,

@@ -79,6 +79,11 @@ cudaError_t launch_build_mask(const MaskArgs& a, cudaStream_t stream);
 int64_t mask_workspace_bytes(int kind, int64_t rows, int64_t nb);
 cudaError_t launch_build_mask_packed(const MaskArgs& a, void* workspace, cudaStream_t stream);
 
+// The packed build with its workspace in the library's own static device array (at most
+// mask_noalloc_scratch_bytes(); the caller checks the size first).
+int64_t mask_noalloc_scratch_bytes();
+cudaError_t launch_build_mask_noalloc(const MaskArgs& a, cudaStream_t stream);
+
 struct AttnArgs {
   const void* q;
   const void* k;

@@ -7,6 +7,7 @@
 //   3. fill:  the count warp's pass again, writing each set column at its ballot rank.
 // Rows come out in (mask head, query block) order with ascending, unique columns, which is
 // a pure function of the parameters: the same CSR on every run.
+#include <atomic>
 #include <cstdint>
 
 #include "kernels.h"
@@ -390,7 +391,39 @@ __global__ void __launch_bounds__(kPackWarps * 32) mask_fill_packed_kernel(const
   }
 }
 
+// Scratch of lva_build_block_mask_noalloc: the workspace of the packed static build, held
+// in the library's own device memory for callers that cannot allocate any.  Every device
+// that loads the library holds the array until the process exits; every call uses all of
+// it that it needs, so calls that overlap on the GPU race.  Nothing in it needs to start at
+// zero: a build writes each scratch byte it reads earlier in the same build.
+constexpr int64_t kNoAllocScratchBytes = int64_t(16) << 20;
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+std::atomic<void*> g_noalloc_ptr[kMaxCachedDevices] = {};
+
+// Device address of the current device's scratch array.  In host code the array's name
+// stands for a host-side shadow, not device memory, so the address is looked up (once per
+// device, with that device current) and passed to the kernels.
+cudaError_t noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cacheable = dev >= 0 && dev < kMaxCachedDevices;
+  if (cacheable) {
+    void* cached = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (cached != nullptr) { *out = cached; return cudaSuccess; }
+  }
+  void* ptr = nullptr;
+  e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  if (ptr == nullptr || (reinterpret_cast<uintptr_t>(ptr) & 255) != 0) return cudaErrorInvalidDevicePointer;
+  if (cacheable) g_noalloc_ptr[dev].store(ptr, std::memory_order_release);
+  *out = ptr;
+  return cudaSuccess;
+}
+
 }  // namespace
+
+int64_t mask_noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
 
 // Workspace: the packed rows (rows x wpr words), the row counts (rows words, scanned in
 // place tile by tile) and the tile sums.
@@ -427,6 +460,17 @@ cudaError_t launch_build_mask_packed(const MaskArgs& a, void* workspace, cudaStr
                                                                   tiles == 1 ? nullptr : sums, a.row_ptr,
                                                                   a.col_idx);
   return cudaGetLastError();
+}
+
+cudaError_t launch_build_mask_noalloc(const MaskArgs& a, cudaStream_t stream) {
+  const int64_t nb = a.n_pad / a.block_size;
+  const int64_t need = mask_workspace_bytes(a.kind, int64_t(a.mask_heads) * nb, nb);
+  if (need == 0) return launch_build_mask(a, stream);
+  if (need > kNoAllocScratchBytes) return cudaErrorInvalidValue;   // checked by the caller first
+  void* scratch = nullptr;
+  const cudaError_t e = noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  return launch_build_mask_packed(a, scratch, stream);
 }
 
 cudaError_t launch_build_mask(const MaskArgs& a, cudaStream_t stream) {

@@ -186,6 +186,32 @@ lva_status lva_build_block_mask_ws(const lva_mask_params* params, const uint8_t*
                                    cudaStream_t stream);
 
 /*
+ * lva_build_block_mask_noalloc -- lva_build_block_mask_ws without a caller workspace.
+ *
+ * An addition of this library; the pages have no counterpart.  For callers that cannot
+ * allocate device memory at all: code that runs inside a host framework which owns every
+ * device allocation and hands its plugins only their input and output buffers, or a
+ * real-time path with a fixed memory budget where no allocation may happen after start-up.
+ * This call builds the same CSR, bit for bit, as lva_build_block_mask_ws, with that call's
+ * workspace taken from a 16 MiB array that the library itself places in device memory: it
+ * calls no cudaMalloc, cudaFree or other allocating routine.  The caller still passes the
+ * mask and the CSR outputs (arguments and errors as for lva_build_block_mask).
+ *
+ * Limit: lva_block_mask_workspace_bytes(params) must be at most 16 MiB (16777216 bytes;
+ * for STATIC masks about 128 Mi block pairs, e.g. 4 heads of 4096 x 4096 blocks), else
+ * LVA_ERR_CAPACITY is returned and nothing is launched.  The parametric kinds need no
+ * scratch.  Every device that loads the library holds the 16 MiB until the process exits.
+ * The first call on a device looks up the array's device address (a runtime call, done once
+ * per device with that device current); make that first call before any stream capture.
+ * All calls share the one array, so calls whose work overlaps on the GPU (other streams,
+ * other host threads) race and must be ordered by the caller; the array keeps the last
+ * call's contents, and a call reads only what it has written itself.
+ */
+lva_status lva_build_block_mask_noalloc(const lva_mask_params* params, const uint8_t* dense_mask,
+                                        int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                                        int32_t* nnz_out, cudaStream_t stream);
+
+/*
  * lva_block_sparse_attn -- softmax attention computed only on listed block pairs.
  *
  * The block-sparse attention of the LVSA page (technical summary section 2: attention
