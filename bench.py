@@ -15,8 +15,10 @@ resident in HBM before the timed region.
   cpu_baseline  the FP64 oracle on a bounded, time-limited sample of the same workload.
 
 ``--impl reference`` times the oracle itself as the reference arm (rank 0 only).
-Multi-GPU (torchrun): every rank runs its own batch element (weak scaling, no collective
-on the data path; a barrier and a max-reduce of the timings only).
+Multi-GPU (torchrun): every rank runs its own batch element (``--shard batch``, weak
+scaling), or one layer is split into contiguous head ranges (``--shard heads``, strong
+scaling, the mask replicated).  Neither has a collective on the data path: a barrier and a
+max-reduce of the timings only.
 """
 from __future__ import annotations
 
@@ -57,7 +59,18 @@ def _workload_for_rank(rank: int) -> Workload:
     return Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
 
 
-def _config_dict(w: Workload, spec: dict, n_gpus: int) -> dict:
+def _config_dict(w: Workload, spec: dict, n_gpus: int, shard: str = "batch") -> dict:
+    if shard == "heads":
+        return {"workload": f"video-DiT-small-like: one layer (B=1, {w.H} heads) split by heads over {n_gpus} GPU(s), "
+                            f"d={w.d}, latent grid {w.T}x{w.Hg}x{w.Wg}={w.n_valid} tokens padded to {w.n_pad}, "
+                            f"tiles 1x8x16, {w.block_size}x{w.block_size} blocks, +-1 latent-frame window + 4 rotating "
+                            f"anchor blocks, denoising step = step index mod 50",
+                "global_batch": w.B, "heads": w.H, "head_dim": w.d, "seq_len": w.n_pad, "block": w.block_size,
+                "step_contents": "per rank, its contiguous head range: reorder of stacked QKV + CSR build (3 "
+                                 "launches, the mask replicated) + attention with the inverse reorder fused into "
+                                 "its epilogue; no collective on the data path",
+                "l2": "inputs larger than L2 at 1-2 GPUs (302 MB Q/K/V in all), no flush",
+                "parallelism": f"heads{n_gpus} (contiguous head ranges of one layer)"}
     return {"workload": f"video-DiT-small-like: B=1 per GPU, {w.H} heads, d={w.d}, latent grid "
                         f"{w.T}x{w.Hg}x{w.Wg}={w.n_valid} tokens padded to {w.n_pad}, tiles 1x8x16, "
                         f"{w.block_size}x{w.block_size} blocks, +-1 latent-frame window + 4 rotating "
@@ -171,17 +184,26 @@ def run_lva(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
-    w = _workload_for_rank(rank)
     spec = mask_variants(WORKLOADS[WORKLOAD])[0]
     n_steps_cycle = len(spec["steps"])
-    q, k, v = make_qkv(w)
+    if args.shard == "heads":
+        # one layer, split into contiguous head ranges: every rank draws only its own heads
+        w = WORKLOADS[WORKLOAD]
+        h0, h1 = lva.head_range(w.H, ws, rank)
+        heads = list(range(h0, h1))
+    else:
+        # every rank its own batch element (its own seed)
+        w = _workload_for_rank(rank)
+        heads = list(range(w.H))
+    H_local = len(heads)
+    q, k, v = make_qkv(w, heads=heads)
     # Q, K, V as one stacked raster buffer (as a fused QKV projection produces them).
     qkv = torch.stack([q, k, v]).to(dev)
     qd, kd, vd = qkv[0], qkv[1], qkv[2]
-    layer = lva.VideoBlockSparseAttention(w.B, w.H, w.d, (w.T, w.Hg, w.Wg), w.tile, w.block_size, spec,
+    layer = lva.VideoBlockSparseAttention(w.B, H_local, w.d, (w.T, w.Hg, w.Wg), w.tile, w.block_size, spec,
                                           scale=w.scale, device=dev)
     nnz = _nnz_table(layer, range(n_steps_cycle))
-    fpn = _flops_per_nnz(w) * w.B * w.H          # mask_heads = 1: every head shares the CSR
+    fpn = _flops_per_nnz(w) * w.B * H_local      # mask_heads = 1: every head shares the CSR
     stream = torch.cuda.current_stream(dev)
 
     def step(kidx, ev=None):
@@ -226,8 +248,8 @@ def run_lva(args):
 
     # ---------------- e2e through the public API with pinned host buffers
     qkvh = torch.stack([q, k, v]).pin_memory()
-    oh = torch.empty((w.B, w.H, w.n_valid, w.d), dtype=torch.bfloat16).pin_memory()
-    lh = torch.empty((w.B, w.H, w.n_pad), dtype=torch.float32).pin_memory()
+    oh = torch.empty((w.B, H_local, w.n_valid, w.d), dtype=torch.bfloat16).pin_memory()
+    lh = torch.empty((w.B, H_local, w.n_pad), dtype=torch.float32).pin_memory()
 
     last_done = [None]
 
@@ -266,9 +288,10 @@ def run_lva(args):
         line = {
             "metric": METRIC, "value": flops_all / (ms_total * 1e-3) / 1e12, "unit": "TFLOP/s",
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": ms_total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": ms_total / args.steps, "higher_is_better": True,
+            "scaling": "strong" if args.shard == "heads" else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16 Q/K/V)",
-            "config": _config_dict(w, spec, ws),
+            "config": _config_dict(w, spec, ws, args.shard),
             "attn_ms_per_layer": attn_ms_mean,
             "active_block_pairs_per_head": {"min": min(nnz.values()), "max": max(nnz.values()),
                                              "density": float(np.mean(list(nnz.values()))) / w.nb ** 2},
@@ -620,6 +643,9 @@ def main():
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="lva", choices=["lva", "reference"])
+    ap.add_argument("--shard", default="batch", choices=["batch", "heads"],
+                    help="batch: every rank its own batch element (weak scaling); heads: one layer split into "
+                         "contiguous head ranges (strong scaling)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

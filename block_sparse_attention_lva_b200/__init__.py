@@ -15,6 +15,7 @@ from ._binding import (LVA_MASK_ALL, LVA_MASK_LVSA_FRAMES, LVA_MASK_STATIC, LVA_
                        lva_device_error, lva_reorder_tokens, lva_select_blocks,
                        lva_selftest_wait, lva_version, lva_layer_step_host)
 from .pipeline import SquadTwoPass, StaticMaskCalibrator, VideoBlockSparseAttention, mask_params_for
+from .sharding import HeadShard, head_range, shard_rows
 
 __all__ = ["LVA_MASK_ALL", "LVA_MASK_LVSA_FRAMES", "LVA_MASK_STATIC", "LVA_MASK_TWO_STAGE", "LVA_MASK_WINDOW_ANCHOR", "LIB_PATH",
            "LvaError", "MaskParams", "lva_block_mask_max_nnz", "lva_block_sparse_attn", "lva_broadcast_blocks",
@@ -23,4 +24,5 @@ __all__ = ["LVA_MASK_ALL", "LVA_MASK_LVSA_FRAMES", "LVA_MASK_STATIC", "LVA_MASK_
            "lva_device_error", "lva_reorder_tokens", "lva_version",
            "lva_block_energy", "lva_select_blocks", "lva_aggregate_masks", "lva_block_sparse_attn_raster", "lva_block_sparse_lse",
            "lva_window_transposed_attn", "lva_selftest_wait", "lva_layer_step_host",
-           "SquadTwoPass", "StaticMaskCalibrator", "VideoBlockSparseAttention", "mask_params_for"]
+           "SquadTwoPass", "StaticMaskCalibrator", "VideoBlockSparseAttention", "mask_params_for",
+           "HeadShard", "head_range", "shard_rows"]
