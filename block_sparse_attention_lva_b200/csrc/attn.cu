@@ -219,6 +219,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     }
   };
 
+  // The producer and issuer warps wait in mbarrier.try_wait (the warp sleeps until the phase
+  // completes), so their waits take no issue slots from the softmax warps that share their
+  // schedulers; the softmax warps poll, since their hand-offs are on the critical path.
+  //
   // A TMA producer: key block T (over all items) goes to slot T % ST of a ring whose slots
   // are released by `empty` barriers; after an abort it waits for the loads still in flight.
   auto produce = [&](const void* tmap, uint32_t ring, int ST, uint32_t full0, uint32_t empty0, int code,
@@ -232,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       if (lane == 0) {
         if (with_q) {
           // Q is single-buffered: the previous item's Q K^T must have completed.
-          if (nq > 0 && !mbar_wait(bar_q_empty, (nq - 1) & 1, abort_flag)) {
+          if (nq > 0 && !mbar_wait_sleep(bar_q_empty, (nq - 1) & 1, abort_flag)) {
             *abort_flag = 1; report_fault(p.err, 5, 8);
           } else {
             mbar_arrive_expect_tx(bar_q, C::Q_BYTES);
@@ -243,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         }
         for (int t = 0; t < w.n && !*abort_flag; ++t, ++T) {
           const int s = int(T % ST);
-          if (T >= ST && !mbar_wait(empty0 + 8u * s, int((T / ST) - 1) & 1, abort_flag)) {
+          if (T >= ST && !mbar_wait_sleep(empty0 + 8u * s, int((T / ST) - 1) & 1, abort_flag)) {
             *abort_flag = 1; report_fault(p.err, 5, code); break;
           }
           const int32_t j = __ldg(p.col_idx + w.start + t);
@@ -287,11 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       const Item w = item_at(it);
       if (w.n == 0) continue;
       if (lane == 0) {
-        ok = mbar_wait(bar_q, nq & 1, abort_flag);
+        ok = mbar_wait_sleep(bar_q, nq & 1, abort_flag);
         for (int t = 0; ok && t < w.n; ++t, ++T) {
           const int s = int(T % C::KST), b = int(T & 1);
-          if (!mbar_wait(bar_k_full(s), int(T / C::KST) & 1, abort_flag)) { ok = false; break; }
-          if (T >= 2 && !mbar_wait(bar_s_free(b), int((T >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_sleep(bar_k_full(s), int(T / C::KST) & 1, abort_flag)) { ok = false; break; }
+          if (T >= 2 && !mbar_wait_sleep(bar_s_free(b), int((T >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ks = k_desc + uint64_t((s * C::KV_BYTES) >> 4);
           const uint32_t s_tm = tmem + C::TM_S + 128 * b;
@@ -332,11 +336,11 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         const Item w = item_at(it);
         if (w.n == 0) continue;
         if (lane == 0) {
-          if (nq > 0) ok = mbar_wait(bar_o_free, (nq - 1) & 1, abort_flag);
+          if (nq > 0) ok = mbar_wait_sleep(bar_o_free, (nq - 1) & 1, abort_flag);
           for (int t = 0; ok && t < w.n; ++t, ++T) {
             const int s = int(T % C::VST), b = int(T & 1);
-            if (!mbar_wait(bar_p_full(b), int(T >> 1) & 1, abort_flag)) { ok = false; break; }
-            if (!mbar_wait(bar_v_full(s), int(T / C::VST) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_sleep(bar_p_full(b), int(T >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_sleep(bar_v_full(s), int(T / C::VST) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
             const uint32_t p_tm = tmem + C::TM_P + 64 * b;
@@ -400,35 +404,40 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_s_free(b));
-        // Real keys of this half (only the block holding the sequence end is partial).  The
-        // choice of path is made for the whole warp: the exponential loop below issues
-        // warp-collective TMEM stores, and the two halves of a row can differ at the end.
-        const int64_t valid = p.n_valid - int64_t(j) * BN - hf * HALF;
-        const bool full = __all_sync(0xffffffffu, valid >= HALF);
-        float mx;
-        if (full) {
+        // Real keys of this half (only the block holding the sequence end is partial).  Scores
+        // of padding keys become a sentinel whose scaled value is -inf (its exponential is 0,
+        // or 2^-125 on the FMA-pipe path: nothing next to a real key's), so one path serves
+        // every block; a block of padding only (possible when n_pad - n_valid >= Bs) stores
+        // P = 0 and adds nothing.  The choice is the whole warp's: the key block is the same
+        // for every lane.
+        const int64_t valid_blk = p.n_valid - int64_t(j) * BN;
+        const bool any_key = valid_blk > 0;
+        if (any_key && valid_blk < BN) {
+          const int64_t valid = valid_blk - hf * HALF;
+          const uint32_t sentinel = __float_as_uint(c >= 0.f ? -INFINITY : INFINITY);
+#pragma unroll
+          for (int e = 0; e < HALF; ++e)
+            if (e >= valid) sr[e] = sentinel;
+        }
+        float mx = -INFINITY;
+        if (any_key) {
           // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (3-input max, 4 chains)
           float m4[4];
           if (c >= 0.f) {
-  #pragma unroll
+#pragma unroll
             for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
-  #pragma unroll
+#pragma unroll
             for (int e = 0; e < HALF / 2; ++e)
               m4[e & 3] = fmax3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
             mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
           } else {
-  #pragma unroll
+#pragma unroll
             for (int e = 0; e < 4; ++e) m4[e] = INFINITY;
-  #pragma unroll
+#pragma unroll
             for (int e = 0; e < HALF / 2; ++e)
               m4[e & 3] = fmin3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
             mx = fminf(fminf(m4[0], m4[1]), fminf(m4[2], m4[3])) * c;
           }
-        } else {
-          mx = -INFINITY;
-  #pragma unroll
-          for (int e = 0; e < HALF; ++e)
-            if (e < valid) mx = fmaxf(mx, __uint_as_float(sr[e]) * c);
         }
         // Row max over both halves (lanes t and t ^ 16 hold one row).
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -447,14 +456,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         const uint32_t p_tm = tmem + lane_off + C::TM_P + 64 * b;
         float r4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[HALF / 2];
-        if (full) {
+        if (any_key) {
           // Pairs of elements with packed fp32 math; every fourth pair takes its exponentials
           // on the FMA pipe, the rest on the MUFU (of 1/2, 1/3, 1/4 and none on the FMA pipe,
           // 1/4 measured fastest).  With 64-key halves the first 16 pairs go to TMEM while the
           // rest are computed.
           const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
           uint64_t acc[2] = {0ull, 0ull};
-  #pragma unroll
+#pragma unroll
           for (int e = 0; e < HALF / 2; ++e) {
             const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
             uint64_t p2;
@@ -486,17 +495,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           f2_unpack(acc[0], a0, a1);
           f2_unpack(acc[1], b0, b1);
           r4[0] = a0; r4[1] = a1; r4[2] = b0; r4[3] = b1;
-        } else {
-  #pragma unroll
-          for (int e = 0; e < HALF; e += 2) {
-            const float p0 = e < valid ? ex2_approx(fmaf(__uint_as_float(sr[e]), c, -m_use)) : 0.f;
-            const float p1 = e + 1 < valid ? ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -m_use)) : 0.f;
-            r4[(e >> 1) & 3] += p0 + p1;
-            pk[e / 2] = pack_bf16x2(p0, p1);
-          }
-          // P half row (bf16 pairs) -> TMEM P_b, the A operand of O += P V.
-          if constexpr (LSE_ONLY) {
-          } else if constexpr (HALF == 64) {
+        } else if constexpr (!LSE_ONLY) {
+#pragma unroll
+          for (int e = 0; e < HALF / 2; ++e) pk[e] = 0u;
+          if constexpr (HALF == 64) {
             tmem_st_16x2_32<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[32]>(pk));
           } else {
             tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
