@@ -32,6 +32,7 @@
 // slice of each row, eight rows per 1024-byte atom.  Q and K are K-major; V is read
 // MN-major straight from its [keys, d] layout; P is the TMEM A operand of P*V.
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -387,13 +388,19 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         report_fault(p.err, 1, (p.mask_heads == 1 ? 0 : w.plane % p.H) * p.nb + w.i);
       float m_ref = -INFINITY;                    // running max in log2 units (lazy)
       float l = 0.f;                              // this half's share of the row sum
-      int32_t jn = n > 0 ? __ldg(p.col_idx + w.start) : 0;
+      // Key blocks j >= n_valid / Bs hold padding keys: the block holding the sequence end and
+      // any block of padding only (possible when n_pad - n_valid >= Bs).  CSR rows ascend, so
+      // they are the row's last entries: entries [0, t_tail) take the step without padding
+      // code, entries [t_tail, n) the masked step.  (Every lane reads the same entries.)
+      const int64_t j_part = p.n_valid / BN;
+      int t_tail = n;
+      while (t_tail > 0 && int64_t(__ldg(p.col_idx + w.start + t_tail - 1)) >= j_part) --t_tail;
 
-      for (int t = 0; t < n; ++t, ++T) {
+      // One key block t (pipeline position T); false when a wait gives up.
+      auto step = [&](int t, auto masked_tag) -> bool {
+        constexpr bool MASKED = decltype(masked_tag)::value;
         const int b = int(T & 1);
-        const int32_t j = jn;
-        if (t + 1 < n) jn = __ldg(p.col_idx + w.start + t + 1);
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T >> 1) & 1, abort_flag))) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T >> 1) & 1, abort_flag))) return false;
         tc_fence_after();
         uint32_t sr[HALF];
 #pragma unroll
@@ -404,20 +411,21 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_s_free(b));
-        // Real keys of this half (only the block holding the sequence end is partial).  Scores
-        // of padding keys become a sentinel whose scaled value is -inf (its exponential is 0,
-        // or 2^-125 on the FMA-pipe path: nothing next to a real key's), so one path serves
-        // every block; a block of padding only (possible when n_pad - n_valid >= Bs) stores
-        // P = 0 and adds nothing.  The choice is the whole warp's: the key block is the same
-        // for every lane.
-        const int64_t valid_blk = p.n_valid - int64_t(j) * BN;
-        const bool any_key = valid_blk > 0;
-        if (any_key && valid_blk < BN) {
-          const int64_t valid = valid_blk - hf * HALF;
-          const uint32_t sentinel = __float_as_uint(c >= 0.f ? -INFINITY : INFINITY);
+        // Masked step: the real keys of this half.  Scores of padding keys become a sentinel
+        // whose scaled value is -inf (its exponential is 0, or 2^-125 on the FMA-pipe path:
+        // nothing next to a real key's); a block of padding only stores P = 0 and adds
+        // nothing.  The choice is the whole warp's: the key block is the same for every lane.
+        bool any_key = true;
+        if constexpr (MASKED) {
+          const int64_t valid_blk = p.n_valid - int64_t(__ldg(p.col_idx + w.start + t)) * BN;
+          any_key = valid_blk > 0;
+          if (any_key) {
+            const int64_t valid = valid_blk - hf * HALF;
+            const uint32_t sentinel = __float_as_uint(c >= 0.f ? -INFINITY : INFINITY);
 #pragma unroll
-          for (int e = 0; e < HALF; ++e)
-            if (e >= valid) sr[e] = sentinel;
+            for (int e = 0; e < HALF; ++e)
+              if (e >= valid) sr[e] = sentinel;
+          }
         }
         float mx = -INFINITY;
         if (any_key) {
@@ -450,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         // phase.  (Almost always complete by now: P(t-2) V was issued a block earlier.)
         if (!LSE_ONLY && T >= 2 &&
             !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), int((T >> 1) - 1) & 1, abort_flag))) {
-          ok = false; break;
+          return false;
         }
         tc_fence_after();
         const uint32_t p_tm = tmem + lane_off + C::TM_P + 64 * b;
@@ -510,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         // before P(t) is released to the P V issuer.
         if (!LSE_ONLY && t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
           if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(b ^ 1), int((T - 1) >> 1) & 1, abort_flag))) {
-            ok = false; break;
+            return false;
           }
           tc_fence_after();
   #pragma unroll 1
@@ -529,7 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_p_full(b));
         }
-      }
+        return true;
+      };
+      for (int t = 0; ok && t < t_tail; ++t, ++T) ok = step(t, std::false_type{});
+      for (int t = t_tail; ok && t < n; ++t, ++T) ok = step(t, std::true_type{});
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue of this item
