@@ -124,7 +124,24 @@ __device__ __forceinline__ int csr_row(const AttnParams& p, int64_t row, int32_t
   return b - a;
 }
 
-template <int D, int BN, int KPC, bool LSE_ONLY>
+// O *= alpha for this thread's half row (the lazy rescale, rare once an item's running max
+// has settled), out of line so that its code and registers stay out of the softmax loop.
+template <int DH>
+__device__ __noinline__ void rescale_o(uint32_t taddr, float alpha) {
+#pragma unroll 1
+  for (int q = 0; q < DH / 32; ++q) {
+    uint32_t ov[32];
+    tmem_ld_16x2_32<DH>(taddr + q * 32, ov);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+    tmem_st_16x2_32<DH>(taddr + q * 32, ov);
+  }
+}
+
+// NEG: the softmax scale is negative, so the row max of scale * s is scale * min(s) (a
+// separate instantiation keeps the positive-scale loop free of that path).
+template <int D, int BN, int KPC, bool LSE_ONLY, bool NEG>
 __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -421,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           any_key = valid_blk > 0;
           if (any_key) {
             const int64_t valid = valid_blk - hf * HALF;
-            const uint32_t sentinel = __float_as_uint(c >= 0.f ? -INFINITY : INFINITY);
+            const uint32_t sentinel = __float_as_uint(NEG ? INFINITY : -INFINITY);
 #pragma unroll
             for (int e = 0; e < HALF; ++e)
               if (e >= valid) sr[e] = sentinel;
@@ -431,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         if (any_key) {
           // max of s*c is c*max(s) for c >= 0 and c*min(s) otherwise (3-input max, 4 chains)
           float m4[4];
-          if (c >= 0.f) {
+          if constexpr (!NEG) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) m4[e] = -INFINITY;
 #pragma unroll
@@ -521,15 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
             return false;
           }
           tc_fence_after();
-  #pragma unroll 1
-          for (int q = 0; q < DH / 32; ++q) {
-            uint32_t ov[32];
-            tmem_ld_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
-            tmem_wait_ld();
-  #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st_16x2_32<DH>(tmem + lane_off + C::TM_O + q * 32, ov);
-          }
+          rescale_o<DH>(tmem + lane_off + C::TM_O, alpha);
         }
         if constexpr (!LSE_ONLY) {
           tmem_wait_st();
@@ -611,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
   }
 }
 
-template <int D, int BN, int KPC, bool LSE_ONLY>
+template <int D, int BN, int KPC, bool LSE_ONLY, bool NEG>
 cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why) {
   using C = Cfg<D, BN, LSE_ONLY>;
   const int64_t rows = int64_t(a.B) * a.H * a.n_pad;
@@ -632,7 +641,7 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   }
   static DeviceFlags attr_set = {};
   cudaError_t e = once_per_device(attr_set, [] {
-    return cudaFuncSetAttribute(bsa_fwd_kernel<D, BN, KPC, LSE_ONLY>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(bsa_fwd_kernel<D, BN, KPC, LSE_ONLY, NEG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 C::SMEM_BYTES);
   });
   if (e != cudaSuccess) { *why = "cudaFuncSetAttribute(max dynamic smem) failed"; return e; }
@@ -659,7 +668,7 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   if (items == 0) return cudaSuccess;
   p.items = items;
   const int64_t grid = (items + KPC - 1) / KPC;
-  bsa_fwd_kernel<D, BN, KPC, LSE_ONLY><<<dim3(unsigned(grid)), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  bsa_fwd_kernel<D, BN, KPC, LSE_ONLY, NEG><<<dim3(unsigned(grid)), kThreads, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -674,10 +683,12 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
 // otherwise 1 (a capacity larger than the entry count therefore selects 1).
 template <int D, int BN, bool LSE_ONLY>
 cudaError_t launch_dispatch(const AttnArgs& a, cudaStream_t stream, const char** why) {
+  // A negative softmax scale (rare) takes its own instantiation, one query block per CTA.
+  if (a.scale < 0.f) return launch_cfg<D, BN, 1, LSE_ONLY, true>(a, stream, why);
   const int64_t rows = int64_t(a.mask_heads) * (a.n_pad / a.block_size);
-  if (rows > 0 && a.col_len <= 3 * rows) return launch_cfg<D, BN, 8, LSE_ONLY>(a, stream, why);
-  if (rows > 0 && a.col_len <= 8 * rows) return launch_cfg<D, BN, 4, LSE_ONLY>(a, stream, why);
-  return launch_cfg<D, BN, 1, LSE_ONLY>(a, stream, why);
+  if (rows > 0 && a.col_len <= 3 * rows) return launch_cfg<D, BN, 8, LSE_ONLY, false>(a, stream, why);
+  if (rows > 0 && a.col_len <= 8 * rows) return launch_cfg<D, BN, 4, LSE_ONLY, false>(a, stream, why);
+  return launch_cfg<D, BN, 1, LSE_ONLY, false>(a, stream, why);
 }
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t stream, const char** why) {

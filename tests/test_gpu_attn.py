@@ -197,6 +197,35 @@ def test_lse_only_matches_attention_lse(B, H, n_pad, n_valid, d, bs, hm, density
     assert np.abs(a[fin] - lse_ref[fin]).max() <= 1e-3
 
 
+
+@pytest.mark.parametrize("d,bs,n_pad,n_valid,seed", [(128, 128, 1280, 1200, 31), (64, 64, 768, 700, 32)])
+def test_negative_scale(d, bs, n_pad, n_valid, seed):
+    """A negative softmax scale (the row max of scale * s is scale * min s) runs its own
+    kernel instantiation: every element of O and LSE, and the LSE-only form, match the
+    oracle; padded keys (scores that would dominate if attended) stay excluded."""
+    import block_sparse_attention_lva_b200 as lva
+    dev = require_gpu()
+    q, k, v = (_rand_bf16((1, 2, n_pad, d), seed + 100 * t) for t in range(3))
+    k[:, :, n_valid:] = -40.0
+    nb = n_pad // bs
+    masks = np.random.default_rng(seed).random((2, nb, nb)) < 0.5
+    masks[0, 0] = False
+    masks[-1, nb - 1] = True
+    scale = -1.0 / math.sqrt(d)
+    o, lse = _attn_gpu(q, k, v, masks, bs, n_valid, scale)
+    o_ref, lse_ref = attention_blocked(q, k, v, masks, bs, n_valid, scale)
+    check_o_lse(o, lse, o_ref, lse_ref, f"negative scale {(n_pad, d, bs)}")
+    rp, ci = dense_to_csr(masks)
+    lse_only = torch.full((1, 2, n_pad), float("nan"), dtype=torch.float32, device=dev)
+    lva.lva_block_sparse_lse(q.to(dev), k.to(dev), lse_only, n_valid, bs, torch.from_numpy(rp).to(dev),
+                             torch.from_numpy(ci).to(dev), 2, scale)
+    torch.cuda.synchronize()
+    assert lva.lva_device_error() == (0, 0)
+    a = lse_only.cpu().numpy()
+    assert np.array_equal(np.isneginf(a), np.isneginf(lse_ref))
+    fin = np.isfinite(lse_ref)
+    assert np.abs(a[fin] - lse_ref[fin]).max() <= 1e-3
+
 # ---------------------------------------------------------------- full workloads
 def _oracle_mask(w, spec, step):
     if spec["kind"] == "window_anchor":
