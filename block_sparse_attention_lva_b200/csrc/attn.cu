@@ -548,7 +548,87 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         }
         return true;
       };
-      for (int t = 0; ok && t < t_tail; ++t, ++T) ok = step(t, std::false_type{});
+
+      // Speculative step for a full key block after the item's first: the exponentials are
+      // taken against the current reference max while the block max is computed alongside,
+      // so no max -> exponentials dependency is on the path.  When some row's block max
+      // exceeds its reference by more than the rescale threshold (rare once the first block
+      // has set it), the block is given up before S or P is released and the max-first step
+      // redoes it; otherwise the results are the max-first step's, bit for bit (same reference,
+      // same arithmetic).  Returns 0 when a wait gives up, 1 when done, 2 for a redo.
+      auto step_spec = [&](int t) -> int {
+        (void)t;
+        const int b = int(T & 1);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T >> 1) & 1, abort_flag))) return 0;
+        tc_fence_after();
+        uint32_t sr[HALF];
+#pragma unroll
+        for (int q = 0; q < HALF / 32; ++q)
+          tmem_ld_16x2_32<HALF>(tmem + lane_off + C::TM_S + 128 * b + q * 32,
+                                *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
+        tmem_wait_ld();
+        if (!LSE_ONLY && T >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), int((T >> 1) - 1) & 1, abort_flag)))
+          return 0;
+        tc_fence_after();
+        const uint32_t p_tm = tmem + lane_off + C::TM_P + 64 * b;
+        const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_ref, -m_ref);
+        uint64_t acc[2] = {0ull, 0ull};
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        uint32_t pk[HALF / 2];
+#pragma unroll
+        for (int e = 0; e < HALF / 2; ++e) {
+          m4[e & 3] = fmax3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
+          const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
+          uint64_t p2;
+          if (e % 4 == 3) {
+            p2 = exp2_poly_f2(x2);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          acc[e & 1] = f2_add(acc[e & 1], p2);
+          if constexpr (!LSE_ONLY) {
+            float p0, p1;
+            f2_unpack(p2, p0, p1);
+            pk[e] = pack_bf16x2(p0, p1);
+            if constexpr (HALF == 64) {
+              if (e == 15) tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+            }
+          }
+        }
+        if constexpr (!LSE_ONLY) {
+          if constexpr (HALF == 64) {
+            tmem_st_16x2_16<HALF / 2>(p_tm + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
+          } else {
+            tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          }
+        }
+        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        if constexpr (!LSE_ONLY) tmem_wait_st();     // a redo's P stores follow these
+        if (__any_sync(0xffffffffu, mx > m_ref + kRescaleThreshold || m_ref == -INFINITY)) return 2;
+        float a0, a1, b0, b1;
+        f2_unpack(acc[0], a0, a1);
+        f2_unpack(acc[1], b0, b1);
+        l = l + ((a0 + a1) + (b0 + b1));
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(bar_s_free(b));
+          if constexpr (!LSE_ONLY) mbar_arrive(bar_p_full(b));
+        }
+        return 1;
+      };
+      for (int t = 0; ok && t < t_tail; ++t, ++T) {
+        int r = 2;
+        if constexpr (!NEG) {
+          if (t > 0) r = step_spec(t);
+        }
+        if (r == 0) ok = false;
+        else if (r == 2) ok = step(t, std::false_type{});
+      }
       for (int t = t_tail; ok && t < n; ++t, ++T) ok = step(t, std::true_type{});
       if (!ok) break;
 
