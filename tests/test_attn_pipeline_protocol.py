@@ -8,7 +8,11 @@ through mbarriers whose waits test a phase *parity*:
 * the Q K^T issuer (warp 1): S_b = Q K^T into TMEM buffer b = T mod 2;
 * the P V issuer (warp 11): O += P_b V, with P_b read from TMEM;
 * the softmax warps (2..9), each owning rows of S, P and O: read S_b, write P_b, rescale
-  O rarely, read O in the epilogue.
+  O rarely, read O in the epilogue.  A key block after an item's first takes the
+  speculative step: S_b read, P_b written, and only then S_b and P_b released together;
+  a warp that gives the block up (its rows' max outgrew the reference) redoes it with the
+  max-first step (S_b read again, released at once, P_b written again, O rescaled), which
+  is also the step of an item's first block.
 
 The LSE-only form (``lva_block_sparse_lse``) runs the same roles without the V producer,
 the P V issuer, P and O: the softmax only reads S_b and releases it.
@@ -23,7 +27,8 @@ The model replays each role's waits, arrivals and buffer accesses in the kernel'
 TMA loads land in any order; each issuer's MMAs complete in issue order, and a
 ``tcgen05.commit`` arrives once every MMA its thread issued before it has completed.  A
 seeded random scheduler runs many item runs (empty items, rows of 1 to 5 key blocks, runs
-of 1, 4 and 8 items, random rescale decisions per warp) under many interleavings and checks:
+of 1, 4 and 8 items, random redo and rescale decisions per warp) under many interleavings
+and checks:
 
 * progress: every run ends, with nothing in flight (no deadlock);
 * no phase aliasing: a wait for phase k starts only when its barrier has completed k or
@@ -45,9 +50,11 @@ WARPS = 3            # softmax warps modelled (8 in the kernel; the protocol is 
 class Model(ProtocolModel):
     issuers = ("qk", "pv")
 
-    def __init__(self, items, rescale, rng, omit=(), lse_only=False):
+    def __init__(self, items, rescale, rng, omit=(), lse_only=False, redo=None, early_sfree=False):
         super().__init__(rng, omit)
         self.items, self.rescale, self.lse_only = items, rescale, lse_only
+        self.redo = redo if redo is not None else (lambda *key: True)
+        self.early_sfree = early_sfree       # a planted mistake: S_b released before a redo
         for name, count in [("q", 1), ("q_empty", 1), ("o_free", WARPS), ("final", 1), ("final_pv", 1)]:
             self.barrier(name, count)
         for s in range(KST):
@@ -151,11 +158,37 @@ class Model(ProtocolModel):
         for it, n in enumerate(self.items):
             for t in range(n):
                 b = T & 1
+                if t >= 1:
+                    # speculative step: P_b written before S_b is released
+                    yield from self.wait(f"s_full{b}", T >> 1, "s_full")
+                    self.buf[f"S{b}w{w}"].begin_read(("s", T))
+                    yield                                    # tcgen05.ld of the S rows
+                    self.buf[f"S{b}w{w}"].end_read()
+                    if self.early_sfree:
+                        self.bar[f"s_free{b}"].arrive()
+                    if not self.lse_only:
+                        if T >= 2:
+                            yield from self.wait(f"o_done{b}", (T >> 1) - 1, "p_reuse")
+                        self.buf[f"P{b}w{w}"].begin_write(("p", T), f"sm{w}")
+                        yield                                # exponentials, tcgen05.st of P
+                        self.buf[f"P{b}w{w}"].end_write()
+                    else:
+                        yield                                # exponentials, sums
+                    if not self.redo(w, it, t):
+                        if not self.early_sfree:
+                            self.bar[f"s_free{b}"].arrive()
+                        if not self.lse_only:
+                            self.bar[f"p_full{b}"].arrive()
+                        T += 1
+                        yield
+                        continue
+                # max-first step: an item's first block, or a block the warp gave up
                 yield from self.wait(f"s_full{b}", T >> 1, "s_full")
                 self.buf[f"S{b}w{w}"].begin_read(("s", T))
                 yield                                        # tcgen05.ld of the S rows
                 self.buf[f"S{b}w{w}"].end_read()
-                self.bar[f"s_free{b}"].arrive()
+                if not (self.early_sfree and t >= 1):
+                    self.bar[f"s_free{b}"].arrive()
                 if self.lse_only:
                     T += 1
                     yield                                    # maxima, exponentials, sums
@@ -184,7 +217,7 @@ class Model(ProtocolModel):
 
 def _run(items, seed, omit=(), lse_only=False):
     rng = random.Random(seed)
-    Model(items, random_decisions(rng, 0.3), rng, omit, lse_only).run()
+    Model(items, random_decisions(rng, 0.3), rng, omit, lse_only, redo=random_decisions(rng, 0.3)).run()
 
 
 @pytest.mark.parametrize("lse_only", [False, True])
@@ -257,3 +290,22 @@ def test_waits_implied_on_the_normal_path(omit):
     for sched in range(200):
         _run([5, 1, 3, 2], seed=sched, omit=(omit,))
         _run([1, 1, 1, 1, 1, 1, 1, 1], seed=sched, omit=(omit,))
+
+
+@pytest.mark.parametrize("lse_only", [False, True])
+def test_speculative_step_must_hold_s_until_it_commits(lse_only):
+    """A speculative step that released S_b right after loading it (as the max-first step
+    does) would let Q K^T(T+2) overwrite S_b while a redo reads it again: some schedule
+    shows the hazard.  The kernel releases S_b only when the block commits, or in the
+    max-first step after the second load."""
+    caught = 0
+    for sched in range(600):
+        rng = random.Random(sched)
+        try:
+            Model([5, 1, 3, 2], random_decisions(rng, 0.3), rng, lse_only=lse_only,
+                  redo=random_decisions(rng, 0.5), early_sfree=True).run()
+        except Hazard:
+            caught += 1
+            if caught >= 3:
+                break
+    assert caught > 0
