@@ -52,6 +52,12 @@ constexpr int kThreads = 32 * (kPVWarp + 1);
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when max grows > 2^8
 constexpr uint32_t kTmemCols = 512;
 
+// Exponential pairs on the FMA-pipe polynomial: one in four with P packing and stores (of
+// 1/2, 1/3, 1/4 and none, 1/4 to 3/8 measured fastest), one in three for the LSE-only form,
+// whose FMA pipe has no P work (3.90 ms against 4.09 ms for one in four, 4.32 for one in two).
+template <bool LSE_ONLY>
+__device__ __forceinline__ constexpr bool kPolyPair(int e) { return LSE_ONLY ? (e % 3 == 2) : (e % 4 == 3); }
+
 struct AttnParams {
   int H, nb, mask_heads;
   int64_t n_pad, n_valid;
@@ -482,17 +488,16 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         float r4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[HALF / 2];
         if (any_key) {
-          // Pairs of elements with packed fp32 math; every fourth pair takes its exponentials
-          // on the FMA pipe, the rest on the MUFU (of 1/2, 1/3, 1/4 and none on the FMA pipe,
-          // 1/4 measured fastest).  With 64-key halves the first 16 pairs go to TMEM while the
-          // rest are computed.
+          // Pairs of elements with packed fp32 math; the pairs kPolyPair picks take their
+          // exponentials on the FMA pipe, the rest on the MUFU.  With 64-key halves the first
+          // 16 pairs go to TMEM while the rest are computed.
           const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_use, -m_use);
           uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
           for (int e = 0; e < HALF / 2; ++e) {
             const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
             uint64_t p2;
-            if (e % 4 == 3) {
+            if (kPolyPair<LSE_ONLY>(e)) {
               p2 = exp2_poly_f2(x2);
             } else {
               float x0, x1;
@@ -581,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           m4[e & 3] = fmax3(m4[e & 3], __uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1]));
           const uint64_t x2 = f2_fma(f2_pack_bits(sr[2 * e], sr[2 * e + 1]), c2, nm2);
           uint64_t p2;
-          if (e % 4 == 3) {
+          if (kPolyPair<LSE_ONLY>(e)) {
             p2 = exp2_poly_f2(x2);
           } else {
             float x0, x1;

@@ -172,8 +172,8 @@ def test_repeated_column_is_reported_not_counted_twice():
     (1, 2, 768, 700, 128, 64, 2, 0.4, 23),
 ])
 def test_lse_only_matches_attention_lse(B, H, n_pad, n_valid, d, bs, hm, density, seed):
-    """lva_block_sparse_lse gives the LSE of lva_block_sparse_attn (same scores, maxima and
-    sums) and matches the oracle; empty rows give -inf."""
+    """lva_block_sparse_lse gives the LSE of lva_block_sparse_attn (same scores and maxima;
+    sums within the exponential split's error) and matches the oracle; empty rows give -inf."""
     import block_sparse_attention_lva_b200 as lva
     dev = require_gpu()
     q, k, v = (_rand_bf16((B, H, n_pad, d), seed + 100 * t) for t in range(3))
@@ -191,7 +191,10 @@ def test_lse_only_matches_attention_lse(B, H, n_pad, n_valid, d, bs, hm, density
     a, b = lse.cpu().numpy(), lse_full.cpu().numpy()
     assert np.array_equal(np.isneginf(a), np.isneginf(b))
     fin = np.isfinite(b)
-    assert np.abs(a[fin] - b[fin]).max() <= 1e-5
+    # The two forms send different exponential pairs to the FMA-pipe polynomial (relative
+    # error <= 7.5e-5, tests/test_exp2_poly.py) and the rest to ex2.approx, so their row sums
+    # differ by at most that relative error and their LSEs by at most ~7.5e-5.
+    assert np.abs(a[fin] - b[fin]).max() <= 1e-4
     _, lse_ref = attention_blocked(q, k, v, masks, bs, n_valid, scale)
     assert np.array_equal(np.isneginf(a), np.isneginf(lse_ref))
     assert np.abs(a[fin] - lse_ref[fin]).max() <= 1e-3
