@@ -288,27 +288,28 @@ __device__ __forceinline__ uint32_t nonzero_bits16(uint4 v) {
   uint32_t m = 0;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    uint32_t t = ((((w[k] & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w[k]) & 0x80808080u) >> 7;   // bits 0, 8, 16, 24
-    t = (t | (t >> 7) | (t >> 14) | (t >> 21)) & 0xFu;
-    m |= t << (4 * k);
+    // bit 7 of each byte = (byte != 0); the product gathers bits 7, 15, 23, 31 into bits
+    // 28..31 (the four partial products land on distinct bit positions: no carries)
+    const uint32_t t = (((w[k] & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | w[k]) & 0x80808080u;
+    m |= ((t * 0x00204081u) >> 28) << (4 * k);
   }
   return m;
 }
 
 constexpr int kPackWarps = 8;
-
-// Static masks, pass 1: one warp per row reads the dense row once (16 bytes per lane) and
-// writes it as bits -- bit j of word j / 32 of the packed row (wpr words, the tail words
-// zero) -- and its count to cnt[row].
+// Static masks, pass 1: one warp per row reads the dense row once (16 bytes per lane, eight
+// loads in flight) and writes it as bits -- bit j of word j / 32 of the packed row (wpr
+// words, the tail words zero) -- and its count to cnt[row].
 __global__ void __launch_bounds__(kPackWarps * 32) mask_pack_kernel(const uint8_t* dense, int64_t rows, int64_t nb,
                                                                   int64_t wpr, uint32_t* packed, int32_t* cnt) {
   const int lane = threadIdx.x & 31;
+  const bool vec = nb % 16 == 0 && (reinterpret_cast<uintptr_t>(dense) & 15) == 0;
   for (int64_t row = int64_t(blockIdx.x) * kPackWarps + (threadIdx.x >> 5); row < rows;
        row += int64_t(gridDim.x) * kPackWarps) {
     const uint8_t* src = dense + row * nb;
     uint32_t* dst = packed + row * wpr;
     int32_t count = 0;
-    if (nb % 16 == 0 && (reinterpret_cast<uintptr_t>(dense) & 15) == 0) {
+    if (vec) {
       // up to 4096 columns per round: all of a lane's loads are issued before any is used
       constexpr int kLoads = 8;
       for (int64_t r0 = 0; r0 < nb; r0 += 512 * kLoads) {
@@ -344,17 +345,19 @@ __global__ void __launch_bounds__(kPackWarps * 32) mask_pack_kernel(const uint8_
 // Static masks, pass 3: one warp per row.  Its CSR offsets come from the tile-local
 // inclusive scan of the counts (cnt) plus the scanned tile sums (sums, absent for a single
 // tile); the warp writes row_ptr[row + 1] and expands the packed bits into ascending column
-// indices, 1024 columns (one word per lane) at a time: each lane writes its set bits into a
-// shared-memory staging run at its exclusive prefix count, then the warp copies the run to
-// col_idx with coalesced stores.  The next round's words are loaded before this round is
-// expanded.
+// indices, 1024 columns (one word per lane) at a time.  Each lane writes its word's set bits
+// (16-bit offsets from the round's first column, two per step) into a shared-memory run at
+// its exclusive prefix count; the run starts `sh` entries in, where sh aligns the run's
+// first column index to 16 bytes in col_idx, so that the warp copies it out with 16-byte
+// stores (4 indices per lane per step; the run's two ends with plain stores).  The next
+// round's words are loaded before this round is expanded.
 __global__ void __launch_bounds__(kPackWarps * 32) mask_fill_packed_kernel(const uint32_t* packed, int64_t rows,
                                                                          int64_t nb, int64_t wpr,
                                                                          const int32_t* cnt, const int32_t* sums,
                                                                          int32_t* row_ptr, int32_t* col_idx) {
-  __shared__ int32_t stage[kPackWarps][1024];
+  __shared__ __align__(16) uint16_t stage[kPackWarps][1024 + 8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int32_t* st = stage[warp];
+  uint16_t* st = stage[warp];
   for (int64_t row = int64_t(blockIdx.x) * kPackWarps + warp; row < rows; row += int64_t(gridDim.x) * kPackWarps) {
     const int64_t tile = row / kScanTile;
     const int32_t off = (sums != nullptr && tile > 0) ? sums[tile - 1] : 0;
@@ -377,14 +380,32 @@ __global__ void __launch_bounds__(kPackWarps * 32) mask_fill_packed_kernel(const
         if (lane >= o) incl += t;
       }
       const int total = __shfl_sync(0xffffffffu, incl, 31);
-      int pos = incl - c;
-      const int32_t col0 = int32_t((w0 + lane) * 32);
+      const int sh = int((reinterpret_cast<uintptr_t>(col_idx + base) >> 2) & 3);
+      int pos = incl - c + sh;
+      const uint32_t off0 = uint32_t(lane) * 32u;          // the word's first column in the round
       while (word != 0u) {
-        st[pos++] = col0 + (__ffs(word) - 1);
-        word &= word - 1u;
+        const uint32_t rest = word & (word - 1u);
+        st[pos] = uint16_t(off0 + uint32_t(__ffs(word) - 1));
+        if (rest != 0u) st[pos + 1] = uint16_t(off0 + uint32_t(__ffs(rest) - 1));
+        pos += rest != 0u ? 2 : 1;
+        word = rest & (rest - 1u);
       }
       __syncwarp();
-      for (int k = lane; k < total; k += 32) col_idx[base + k] = st[k];
+      const int32_t col0 = int32_t(w0 * 32);
+      const int end = total + sh;                          // run entries [sh, end) -> col_idx[base ...]
+      for (int c4 = lane * 4; c4 < end; c4 += 128) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(st + c4);
+        const int32_t v0 = col0 + int32_t(raw.x & 0xffffu), v1 = col0 + int32_t(raw.x >> 16);
+        const int32_t v2 = col0 + int32_t(raw.y & 0xffffu), v3 = col0 + int32_t(raw.y >> 16);
+        if (c4 >= sh && c4 + 4 <= end) {
+          *reinterpret_cast<int4*>(col_idx + base + (c4 - sh)) = make_int4(v0, v1, v2, v3);
+        } else {
+          if (c4 >= sh && c4 < end) col_idx[base + (c4 - sh)] = v0;
+          if (c4 + 1 >= sh && c4 + 1 < end) col_idx[base + (c4 + 1 - sh)] = v1;
+          if (c4 + 2 >= sh && c4 + 2 < end) col_idx[base + (c4 + 2 - sh)] = v2;
+          if (c4 + 3 >= sh && c4 + 3 < end) col_idx[base + (c4 + 3 - sh)] = v3;
+        }
+      }
       __syncwarp();
       base += total;
     }
