@@ -229,6 +229,47 @@ def test_negative_scale(d, bs, n_pad, n_valid, seed):
     fin = np.isfinite(lse_ref)
     assert np.abs(a[fin] - lse_ref[fin]).max() <= 1e-3
 
+
+@pytest.mark.parametrize("d,bs,grow_rows", [(128, 128, "all"), (128, 128, "some"), (64, 64, "some")])
+def test_running_max_jumps_take_the_redo_path(d, bs, grow_rows):
+    """Key blocks after a row's first whose scores exceed the running reference by far more
+    than the lazy-rescale threshold: the speculative step must give the block up and the
+    max-first step redo it (with the O rescale).  Every element of O and LSE, and the
+    LSE-only form, match the oracle -- for jumps in every row, and in some rows only (so
+    that some warps redo a block and others commit it)."""
+    import block_sparse_attention_lva_b200 as lva
+    dev = require_gpu()
+    B, H, n_pad, n_valid = 1, 2, 8 * bs, 8 * bs - 9
+    q, k, v = (_rand_bf16((B, H, n_pad, d), 700 + t) for t in range(3))
+    nb = n_pad // bs
+    # Queries share a component along a unit vector u, and the keys of blocks 3 and 6 carry a
+    # large multiple of u: in (nearly) every row the block max of scale * s grows by more
+    # than 8 in log2 units at block 3 and again at block 6.  With "some", only the queries of
+    # even 16-row groups carry the component.
+    u = torch.randn(d, generator=torch.Generator().manual_seed(77))
+    u = u / u.norm()
+    cq = torch.full((n_pad,), 4.0)
+    if grow_rows == "some":
+        cq[(torch.arange(n_pad) // 16) % 2 == 1] = 0.0
+    q = (q.float() + cq[None, None, :, None] * u).to(torch.bfloat16)
+    for jb, amp in ((3, 3.0), (6, 6.0)):
+        k[:, :, jb * bs:(jb + 1) * bs] = (k[:, :, jb * bs:(jb + 1) * bs].float() + amp * math.sqrt(d) * u).to(torch.bfloat16)
+    masks = np.ones((1, nb, nb), dtype=bool)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = _attn_gpu(q, k, v, masks, bs, n_valid, scale)
+    o_ref, lse_ref = attention_blocked(q, k, v, masks, bs, n_valid, scale)
+    check_o_lse(o, lse, o_ref, lse_ref, f"max jumps {(d, bs, grow_rows)}")
+    rp, ci = dense_to_csr(masks)
+    lse_only = torch.full((B, H, n_pad), float("nan"), dtype=torch.float32, device=dev)
+    lva.lva_block_sparse_lse(q.to(dev), k.to(dev), lse_only, n_valid, bs, torch.from_numpy(rp).to(dev),
+                             torch.from_numpy(ci).to(dev), 1, scale)
+    torch.cuda.synchronize()
+    assert lva.lva_device_error() == (0, 0)
+    a = lse_only.cpu().numpy()
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(a), fin)
+    assert np.abs(a[fin] - lse_ref[fin]).max() <= 1e-3
+
 # ---------------------------------------------------------------- full workloads
 def _oracle_mask(w, spec, step):
     if spec["kind"] == "window_anchor":
