@@ -10,16 +10,18 @@
 // fused into the epilogue); Q/K/V rows come from plane-major 2D tensor maps, or from 3D
 // maps that gather the window-transposed order in place (the SQuad page's global pass).
 //
-// Pipeline: S and P are double-buffered in TMEM (S_0, S_1, P_0, P_1, O = 512 columns), so
-// the MMA issuer computes S(t+2) = Q K_{t+2}^T as soon as the softmax has read S(t), and
-// O += P(t) V_t runs while the softmax works on block t+1: the softmax is the only serial
-// chain.
+// Pipeline: three S buffers in TMEM (S_0, S_1, S_2, O = 512 columns).  The softmax writes
+// P(t) as bf16 over the first columns of S(t), which O += P(t) V_t then reads, so buffer
+// t mod 3 is free again once that P V has completed.  The MMA issuer computes S(t+3) =
+// Q K_{t+3}^T then, O += P(t) V_t runs while the softmax works on block t+1, and the softmax
+// never waits for a P buffer: it is the only serial chain.  (The LSE-only form has no P and
+// keeps two S buffers, released as soon as the softmax has read them.)
 //
 // Warp roles (384 threads):
 //   warp 0       TMA producer: Q tile once, then K_j tiles into a 3-slot ring;
 //   warp 10      TMA producer: V_j tiles into a 3-slot ring;
 //   warp 1       MMA issuer (one thread): S_b = Q K_j^T; owns TMEM;
-//   warp 11      MMA issuer (one thread): O += P_b V_j (P_b read from TMEM);
+//   warp 11      MMA issuer (one thread): O += P_b V_j (P_b read from TMEM, over S_b);
 //   warps 2..9   softmax + epilogue: each warp owns 16 rows of the 128-row tile; lane t and
 //                lane t + 16 hold the left and right column halves of one row (the .16x32bx2
 //                TMEM shapes), so row maxima and sums meet through one shuffle; O is
@@ -81,6 +83,10 @@ struct AttnParams {
 template <int D, int BN, bool LSE_ONLY>
 struct Cfg {
   static constexpr int KST = 3, VST = LSE_ONLY ? 0 : 3;
+  // S buffers in TMEM.  With P V, P(t) is written over S(t)'s first columns, so a buffer is
+  // free again once O += P(t) V has completed, and three buffers fit next to O; the LSE-only
+  // form has no P and keeps two, released as soon as the softmax has read them.
+  static constexpr int NSB = LSE_ONLY ? 2 : 3;
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int KV_BYTES = BN * D * 2;
   static constexpr int OFF_Q = 0;
@@ -92,16 +98,16 @@ struct Cfg {
   // q_empty (an item's Q K^T done: Q may be replaced), o_free (an item's O read: P V may
   // start the next item)
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST, B_VE = B_VF + VST,
-                       B_SF = B_VE + VST, B_SE = B_SF + 2, B_P = B_SE + 2, B_O = B_P + 2,
-                       B_FIN = B_O + 2, B_FIN_PV = B_FIN + 1, B_QE = B_FIN_PV + 1, B_OF = B_QE + 1,
+                       B_SF = B_VE + VST, B_SE = B_SF + NSB, B_P = B_SE + NSB, B_O = B_P + NSB,
+                       B_FIN = B_O + NSB, B_FIN_PV = B_FIN + 1, B_QE = B_FIN_PV + 1, B_OF = B_QE + 1,
                        NUM_BARS = B_OF + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // At least 120 KB so that one CTA (and one 512-column TMEM allocation) is resident per SM.
   static constexpr int SMEM_RAW = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
-  // TMEM columns: S_b at 128 b, P_b (bf16 pairs) at 256 + 64 b, O at 384
-  static constexpr uint32_t TM_S = 0, TM_P = 256, TM_O = 384;
+  // TMEM columns: S_b at 128 b (P_b, bf16 pairs, over its first 64 columns), O at 384
+  static constexpr uint32_t TM_S = 0, TM_O = 384;
   static_assert(D <= 128 && BN <= 128, "TMEM layout");
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);
@@ -211,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
     mbar_init(bar_q_empty, 1);
     for (int s = 0; s < C::KST; ++s) { mbar_init(bar_k_full(s), 1); mbar_init(bar_k_empty(s), 1); }
     for (int s = 0; s < C::VST; ++s) { mbar_init(bar_v_full(s), 1); mbar_init(bar_v_empty(s), 1); }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::NSB; ++b) {
       mbar_init(bar_s_full(b), 1);
       mbar_init(bar_s_free(b), kSoftmaxWarps);
       mbar_init(bar_p_full(b), kSoftmaxWarps);
@@ -317,9 +323,14 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       if (lane == 0) {
         ok = mbar_wait_sleep(bar_q, nq & 1, abort_flag);
         for (int t = 0; ok && t < w.n; ++t, ++T) {
-          const int s = int(T % C::KST), b = int(T & 1);
+          const int s = int(T % C::KST), b = int(T % C::NSB);
           if (!mbar_wait_sleep(bar_k_full(s), int(T / C::KST) & 1, abort_flag)) { ok = false; break; }
-          if (T >= 2 && !mbar_wait_sleep(bar_s_free(b), int((T >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+          // S_b is free again: read by the softmax (LSE only), or read and overwritten with P
+          // and that P read by O += P V (the P V of position T - NSB)
+          if (T >= uint32_t(C::NSB) &&
+              !mbar_wait_sleep(LSE_ONLY ? bar_s_free(b) : bar_o_done(b), int((T / C::NSB) - 1) & 1, abort_flag)) {
+            ok = false; break;
+          }
           tc_fence_after();
           const uint64_t ks = k_desc + uint64_t((s * C::KV_BYTES) >> 4);
           const uint32_t s_tm = tmem + C::TM_S + 128 * b;
@@ -362,12 +373,12 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         if (lane == 0) {
           if (nq > 0) ok = mbar_wait_sleep(bar_o_free, (nq - 1) & 1, abort_flag);
           for (int t = 0; ok && t < w.n; ++t, ++T) {
-            const int s = int(T % C::VST), b = int(T & 1);
-            if (!mbar_wait_sleep(bar_p_full(b), int(T >> 1) & 1, abort_flag)) { ok = false; break; }
+            const int s = int(T % C::VST), b = int(T % C::NSB);
+            if (!mbar_wait_sleep(bar_p_full(b), int(T / C::NSB) & 1, abort_flag)) { ok = false; break; }
             if (!mbar_wait_sleep(bar_v_full(s), int(T / C::VST) & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint64_t vs = v_desc + uint64_t((s * C::KV_BYTES) >> 4);
-            const uint32_t p_tm = tmem + C::TM_P + 64 * b;
+            const uint32_t p_tm = tmem + C::TM_S + 128 * b;
   #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
               umma_f16_ts(tmem + C::TM_O, p_tm + kk * 8, vs + uint64_t((kk * 16 * 128) >> 4), C::IDESC_PV,
@@ -422,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       // One key block t (pipeline position T); false when a wait gives up.
       auto step = [&](int t, auto masked_tag) -> bool {
         constexpr bool MASKED = decltype(masked_tag)::value;
-        const int b = int(T & 1);
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T >> 1) & 1, abort_flag))) return false;
+        const int b = int(T % C::NSB);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T / C::NSB) & 1, abort_flag))) return false;
         tc_fence_after();
         uint32_t sr[HALF];
 #pragma unroll
@@ -431,9 +442,11 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           tmem_ld_16x2_32<HALF>(tmem + lane_off + C::TM_S + 128 * b + q * 32,
                                 *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_s_free(b));
+        if constexpr (LSE_ONLY) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_s_free(b));
+        }
         // Masked step: the real keys of this half.  Scores of padding keys become a sentinel
         // whose scaled value is -inf (its exponential is 0, or 2^-125 on the FMA-pipe path:
         // nothing next to a real key's); a block of padding only stores P = 0 and adds
@@ -476,15 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         if (mx > m_ref + kRescaleThreshold || m_ref == -INFINITY) m_ref = fmaxf(mx, m_ref);
         const float alpha = (m_old == m_ref) ? 1.f : ex2_approx(m_old - m_ref);
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // P_b was last read by O += P(t-2) V; wait for it before any part of P(t) is stored.
-        // Each P buffer has its own completion barrier, so the wait never aliases an older
-        // phase.  (Almost always complete by now: P(t-2) V was issued a block earlier.)
-        if (!LSE_ONLY && T >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), int((T >> 1) - 1) & 1, abort_flag))) {
-          return false;
-        }
-        tc_fence_after();
-        const uint32_t p_tm = tmem + lane_off + C::TM_P + 64 * b;
+        // P(t) goes over S(t)'s first columns, which every lane of the warp has loaded (the
+        // row-max shuffle above follows each lane's load wait).
+        __syncwarp();
+        const uint32_t p_tm = tmem + lane_off + C::TM_S + 128 * b;
         float r4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t pk[HALF / 2];
         if (any_key) {
@@ -539,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         // O was last written by O += P(t-1) V: rescale it (rarely) once that has completed,
         // before P(t) is released to the P V issuer.
         if (!LSE_ONLY && t >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(b ^ 1), int((T - 1) >> 1) & 1, abort_flag))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(int((T - 1) % C::NSB)), int((T - 1) / C::NSB) & 1, abort_flag))) {
             return false;
           }
           tc_fence_after();
@@ -563,8 +571,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
       // same arithmetic).  Returns 0 when a wait gives up, 1 when done, 2 for a redo.
       auto step_spec = [&](int t) -> int {
         (void)t;
-        const int b = int(T & 1);
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T >> 1) & 1, abort_flag))) return 0;
+        const int b = int(T % C::NSB);
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full(b), int(T / C::NSB) & 1, abort_flag))) return 0;
         tc_fence_after();
         uint32_t sr[HALF];
 #pragma unroll
@@ -572,11 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
           tmem_ld_16x2_32<HALF>(tmem + lane_off + C::TM_S + 128 * b + q * 32,
                                 *reinterpret_cast<uint32_t(*)[32]>(sr + q * 32));
         tmem_wait_ld();
-        if (!LSE_ONLY && T >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(bar_o_done(b), int((T >> 1) - 1) & 1, abort_flag)))
-          return 0;
-        tc_fence_after();
-        const uint32_t p_tm = tmem + lane_off + C::TM_P + 64 * b;
+        const uint32_t p_tm = tmem + lane_off + C::TM_S + 128 * b;
         const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m_ref, -m_ref);
         uint64_t acc[2] = {0ull, 0ull};
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -598,22 +602,20 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
             float p0, p1;
             f2_unpack(p2, p0, p1);
             pk[e] = pack_bf16x2(p0, p1);
-            if constexpr (HALF == 64) {
-              if (e == 15) tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
-            }
-          }
-        }
-        if constexpr (!LSE_ONLY) {
-          if constexpr (HALF == 64) {
-            tmem_st_16x2_16<HALF / 2>(p_tm + 16, *reinterpret_cast<const uint32_t(*)[16]>(pk + 16));
-          } else {
-            tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
           }
         }
         float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * c;
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        if constexpr (!LSE_ONLY) tmem_wait_st();     // a redo's P stores follow these
+        // A redo reloads S, so P (which goes over S) is stored only once the block commits.
         if (__any_sync(0xffffffffu, mx > m_ref + kRescaleThreshold || m_ref == -INFINITY)) return 2;
+        if constexpr (!LSE_ONLY) {
+          if constexpr (HALF == 64) {
+            tmem_st_16x2_32<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+          } else {
+            tmem_st_16x2_16<HALF / 2>(p_tm, *reinterpret_cast<const uint32_t(*)[16]>(pk));
+          }
+          tmem_wait_st();
+        }
         float a0, a1, b0, b1;
         f2_unpack(acc[0], a0, a1);
         f2_unpack(acc[1], b0, b1);
@@ -621,8 +623,8 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(bar_s_free(b));
-          if constexpr (!LSE_ONLY) mbar_arrive(bar_p_full(b));
+          if constexpr (LSE_ONLY) mbar_arrive(bar_s_free(b));
+          else mbar_arrive(bar_p_full(b));
         }
         return 1;
       };
@@ -659,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
         const float inv_l = have ? 1.f / l_row : 0.f;
         if (n > 0) {
           const uint32_t T_last = T - 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(int(T_last & 1)), int(T_last >> 1) & 1, abort_flag))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done(int(T_last % C::NSB)), int(T_last / C::NSB) & 1, abort_flag))) {
             ok = false; break;
           }
           tc_fence_after();

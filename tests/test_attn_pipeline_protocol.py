@@ -5,23 +5,25 @@ through mbarriers whose waits test a phase *parity*:
 
 * the Q/K producer (warp 0): Q once per item, then K tiles into a 3-slot ring;
 * the V producer (warp 10): V tiles into a 3-slot ring;
-* the Q K^T issuer (warp 1): S_b = Q K^T into TMEM buffer b = T mod 2;
-* the P V issuer (warp 11): O += P_b V, with P_b read from TMEM;
-* the softmax warps (2..9), each owning rows of S, P and O: read S_b, write P_b, rescale
-  O rarely, read O in the epilogue.  A key block after an item's first takes the
-  speculative step: S_b read, P_b written, and only then S_b and P_b released together;
-  a warp that gives the block up (its rows' max outgrew the reference) redoes it with the
-  max-first step (S_b read again, released at once, P_b written again, O rescaled), which
-  is also the step of an item's first block.
+* the Q K^T issuer (warp 1): S_b = Q K^T into TMEM buffer b = T mod 3, once O += P V of
+  position T - 3 (which read P from that buffer) has completed;
+* the P V issuer (warp 11): O += P_b V, with P_b read from TMEM over the first columns of S_b;
+* the softmax warps (2..9), each owning rows of S, P and O: read S_b, write P_b over it,
+  rescale O rarely, read O in the epilogue.  A key block after an item's first takes the
+  speculative step: S_b read, and P_b written only once the block commits; a warp that
+  gives the block up (its rows' max outgrew the reference) redoes it with the max-first
+  step (S_b read again, P_b written, O rescaled), which is also the step of an item's first
+  block.
 
 The LSE-only form (``lva_block_sparse_lse``) runs the same roles without the V producer,
-the P V issuer, P and O: the softmax only reads S_b and releases it.
+the P V issuer, P and O, with two S buffers: the softmax only reads S_b and releases it
+(s_free), and the Q K^T issuer waits for that release.
 
-Positions T count key blocks over all the items a CTA walks, so ring slots (T mod 3), S/P
-buffers (T mod 2) and barrier phases continue from one item to the next; ``q_empty`` and
-``o_free`` hand the single Q tile and the O accumulator from one item to the next.  Items
-with no key blocks (empty rows, corrupt rows, blocks skipped for repetitive heads) take
-no part in the pipeline.
+Positions T count key blocks over all the items a CTA walks, so ring slots (T mod 3), S
+buffers (T mod 3, or T mod 2) and barrier phases continue from one item to the next;
+``q_empty`` and ``o_free`` hand the single Q tile and the O accumulator from one item to the
+next.  Items with no key blocks (empty rows, corrupt rows, blocks skipped for repetitive
+heads) take no part in the pipeline.
 
 The model replays each role's waits, arrivals and buffer accesses in the kernel's order.
 TMA loads land in any order; each issuer's MMAs complete in issue order, and a
@@ -33,9 +35,9 @@ and checks:
 * progress: every run ends, with nothing in flight (no deadlock);
 * no phase aliasing: a wait for phase k starts only when its barrier has completed k or
   k + 1 phases and ends at exactly k + 1 (a parity test cannot tell k from k + 2);
-* no buffer hazard: a K/V ring slot, Q, or a warp's rows of S_b, P_b or O are written only
-  when no read of them is in flight (writes by one MMA issuer may overlap: its MMAs run in
-  order), and read only once written, with the content the reader expects.
+* no buffer hazard: a K/V ring slot, Q, or a warp's rows of S_b (or the P over it) or O are
+  written only when no read of them is in flight (writes by one MMA issuer may overlap: its
+  MMAs run in order), and read only once written, with the content the reader expects.
 """
 import random
 
@@ -50,11 +52,14 @@ WARPS = 3            # softmax warps modelled (8 in the kernel; the protocol is 
 class Model(ProtocolModel):
     issuers = ("qk", "pv")
 
-    def __init__(self, items, rescale, rng, omit=(), lse_only=False, redo=None, early_sfree=False):
+    def __init__(self, items, rescale, rng, omit=(), lse_only=False, redo=None, early_p=False):
         super().__init__(rng, omit)
         self.items, self.rescale, self.lse_only = items, rescale, lse_only
         self.redo = redo if redo is not None else (lambda *key: True)
-        self.early_sfree = early_sfree       # a planted mistake: S_b released before a redo
+        # a planted mistake: the speculative step releases S_b (LSE only) or writes P_b over
+        # it (with P V) before it knows whether the block is redone
+        self.early_p = early_p
+        self.nsb = 2 if lse_only else 3
         for name, count in [("q", 1), ("q_empty", 1), ("o_free", WARPS), ("final", 1), ("final_pv", 1)]:
             self.barrier(name, count)
         for s in range(KST):
@@ -63,15 +68,14 @@ class Model(ProtocolModel):
         for s in range(VST):
             self.barrier(f"v_full{s}", 1)
             self.barrier(f"v_empty{s}", 1)
-        for b in range(2):
+        for b in range(self.nsb):
             for name, count in [("s_full", 1), ("s_free", WARPS), ("p_full", WARPS), ("o_done", 1)]:
                 self.barrier(f"{name}{b}", count)
         for name in ["Q"] + [f"K{s}" for s in range(KST)] + [f"V{s}" for s in range(VST)]:
             self.buffer(name)
         for w in range(WARPS):
-            for b in range(2):
-                self.buffer(f"S{b}w{w}")
-                self.buffer(f"P{b}w{w}")
+            for b in range(self.nsb):
+                self.buffer(f"S{b}w{w}")             # S_b, and P_b over its first columns
             self.buffer(f"Ow{w}")
 
     def roles(self):
@@ -116,10 +120,12 @@ class Model(ProtocolModel):
                 continue
             yield from self.wait("q", nq, "q_full")
             for _ in range(n):
-                s, b = T % KST, T & 1
+                s, b = T % KST, T % self.nsb
                 yield from self.wait(f"k_full{s}", T // KST, "k_full")
-                if T >= 2:
-                    yield from self.wait(f"s_free{b}", (T >> 1) - 1, "s_free")
+                if T >= self.nsb:
+                    # S_b is free: released by the softmax (LSE only), or its P read by P V
+                    free = f"s_free{b}" if self.lse_only else f"o_done{b}"
+                    yield from self.wait(free, T // self.nsb - 1, "s_free")
                 self.issue_mma("qk", [("Q", ("q", it)), (f"K{s}", ("k", T))],
                                [(f"S{b}w{w}", ("s", T), None) for w in range(WARPS)])
                 self.commit("qk", f"s_full{b}")
@@ -139,11 +145,11 @@ class Model(ProtocolModel):
             if nq > 0:
                 yield from self.wait("o_free", nq - 1, "o_free")       # the previous item's O was read
             for t in range(n):
-                s, b = T % VST, T & 1
-                yield from self.wait(f"p_full{b}", T >> 1, "p_full")
+                s, b = T % VST, T % self.nsb
+                yield from self.wait(f"p_full{b}", T // self.nsb, "p_full")
                 yield from self.wait(f"v_full{s}", T // VST, "v_full")
                 o_writes = [(f"Ow{w}", ("o", T), ("o", T - 1) if t > 0 else None) for w in range(WARPS)]
-                self.issue_mma("pv", [(f"P{b}w{w}", ("p", T)) for w in range(WARPS)] + [(f"V{s}", ("v", T))],
+                self.issue_mma("pv", [(f"S{b}w{w}", ("p", T)) for w in range(WARPS)] + [(f"V{s}", ("v", T))],
                                o_writes)
                 self.commit("pv", f"v_empty{s}")
                 self.commit("pv", f"o_done{b}")
@@ -155,51 +161,53 @@ class Model(ProtocolModel):
 
     def softmax(self, w):
         T = 0
+        nsb = self.nsb
         for it, n in enumerate(self.items):
             for t in range(n):
-                b = T & 1
+                b = T % nsb
+                S = f"S{b}w{w}"
                 if t >= 1:
-                    # speculative step: P_b written before S_b is released
-                    yield from self.wait(f"s_full{b}", T >> 1, "s_full")
-                    self.buf[f"S{b}w{w}"].begin_read(("s", T))
+                    # speculative step: P_b (over S_b) written only once the block commits
+                    yield from self.wait(f"s_full{b}", T // nsb, "s_full")
+                    self.buf[S].begin_read(("s", T))
                     yield                                    # tcgen05.ld of the S rows
-                    self.buf[f"S{b}w{w}"].end_read()
-                    if self.early_sfree:
-                        self.bar[f"s_free{b}"].arrive()
-                    if not self.lse_only:
-                        if T >= 2:
-                            yield from self.wait(f"o_done{b}", (T >> 1) - 1, "p_reuse")
-                        self.buf[f"P{b}w{w}"].begin_write(("p", T), f"sm{w}")
-                        yield                                # exponentials, tcgen05.st of P
-                        self.buf[f"P{b}w{w}"].end_write()
-                    else:
-                        yield                                # exponentials, sums
-                    if not self.redo(w, it, t):
-                        if not self.early_sfree:
+                    self.buf[S].end_read()
+                    if self.early_p:
+                        if self.lse_only:
                             self.bar[f"s_free{b}"].arrive()
-                        if not self.lse_only:
+                        else:
+                            self.buf[S].write(("p", T), f"sm{w}")
+                    yield                                    # exponentials (and sums)
+                    if not self.redo(w, it, t):
+                        if self.lse_only:
+                            if not self.early_p:
+                                self.bar[f"s_free{b}"].arrive()
+                        else:
+                            if not self.early_p:
+                                self.buf[S].begin_write(("p", T), f"sm{w}")
+                                yield                        # tcgen05.st of P over S
+                                self.buf[S].end_write()
                             self.bar[f"p_full{b}"].arrive()
                         T += 1
                         yield
                         continue
                 # max-first step: an item's first block, or a block the warp gave up
-                yield from self.wait(f"s_full{b}", T >> 1, "s_full")
-                self.buf[f"S{b}w{w}"].begin_read(("s", T))
+                yield from self.wait(f"s_full{b}", T // nsb, "s_full")
+                self.buf[S].begin_read(("s", T))
                 yield                                        # tcgen05.ld of the S rows
-                self.buf[f"S{b}w{w}"].end_read()
-                if not (self.early_sfree and t >= 1):
-                    self.bar[f"s_free{b}"].arrive()
+                self.buf[S].end_read()
                 if self.lse_only:
+                    if not (self.early_p and t >= 1):
+                        self.bar[f"s_free{b}"].arrive()
                     T += 1
                     yield                                    # maxima, exponentials, sums
                     continue
-                if T >= 2:
-                    yield from self.wait(f"o_done{b}", (T >> 1) - 1, "p_reuse")   # P V(T-2) has read P_b
-                self.buf[f"P{b}w{w}"].begin_write(("p", T), f"sm{w}")
-                yield                                        # exponentials, tcgen05.st of P
-                self.buf[f"P{b}w{w}"].end_write()
+                self.buf[S].begin_write(("p", T), f"sm{w}")
+                yield                                        # exponentials, tcgen05.st of P over S
+                self.buf[S].end_write()
                 if t >= 1 and self.rescale(w, it, t):
-                    yield from self.wait(f"o_done{b ^ 1}", (T - 1) >> 1, "rescale")   # P V(T-1) is done
+                    pb = (T - 1) % nsb
+                    yield from self.wait(f"o_done{pb}", (T - 1) // nsb, "rescale")   # P V(T-1) is done
                     self.buf[f"Ow{w}"].begin_write(("o", T - 1), f"sm{w}", ("o", T - 1))
                     yield                                    # O rows scaled in TMEM
                     self.buf[f"Ow{w}"].end_write()
@@ -207,7 +215,7 @@ class Model(ProtocolModel):
                 T += 1
                 yield
             if n > 0 and not self.lse_only:
-                yield from self.wait(f"o_done{(T - 1) & 1}", (T - 1) >> 1, "epilogue")
+                yield from self.wait(f"o_done{(T - 1) % nsb}", (T - 1) // nsb, "epilogue")
                 self.buf[f"Ow{w}"].begin_read(("o", T - 1))
                 yield                                        # tcgen05.ld of the O rows
                 self.buf[f"Ow{w}"].end_read()
@@ -246,7 +254,7 @@ def test_edge_item_runs(items):
 # Each of these waits is needed on the normal path: without it (in the model only) some
 # schedule breaks a check.
 WAITS = ["q_empty", "k_empty", "v_empty", "q_full", "k_full", "s_free", "p_full", "v_full",
-         "s_full", "p_reuse", "rescale", "epilogue"]
+         "s_full", "rescale", "epilogue"]
 
 
 WAITS_LSE = ["q_empty", "k_empty", "q_full", "k_full", "s_free", "s_full"]
@@ -294,16 +302,16 @@ def test_waits_implied_on_the_normal_path(omit):
 
 @pytest.mark.parametrize("lse_only", [False, True])
 def test_speculative_step_must_hold_s_until_it_commits(lse_only):
-    """A speculative step that released S_b right after loading it (as the max-first step
-    does) would let Q K^T(T+2) overwrite S_b while a redo reads it again: some schedule
-    shows the hazard.  The kernel releases S_b only when the block commits, or in the
-    max-first step after the second load."""
+    """A speculative step that released S_b (LSE only) or wrote P_b over it before knowing
+    whether the block is redone would let a redo read something other than S: Q K^T(T+2)'s
+    result, or P.  Some schedule shows the hazard.  The kernel writes P and releases S_b only
+    once the block commits, or in the max-first step."""
     caught = 0
     for sched in range(600):
         rng = random.Random(sched)
         try:
             Model([5, 1, 3, 2], random_decisions(rng, 0.3), rng, lse_only=lse_only,
-                  redo=random_decisions(rng, 0.5), early_sfree=True).run()
+                  redo=random_decisions(rng, 0.5), early_p=True).run()
         except Hazard:
             caught += 1
             if caught >= 3:
