@@ -16,11 +16,11 @@ through mbarriers whose waits test a phase *parity*:
   block.
 
 The LSE-only form (``lva_block_sparse_lse``) runs the same roles without the V producer,
-the P V issuer, P and O, with two S buffers: the softmax only reads S_b and releases it
+the P V issuer, P and O, with four S buffers: the softmax only reads S_b and releases it
 (s_free), and the Q K^T issuer waits for that release.
 
 Positions T count key blocks over all the items a CTA walks, so ring slots (T mod 3), S
-buffers (T mod 3, or T mod 2) and barrier phases continue from one item to the next;
+buffers (T mod 3, or T mod 4) and barrier phases continue from one item to the next;
 ``q_empty`` and ``o_free`` hand the single Q tile and the O accumulator from one item to the
 next.  Items with no key blocks (empty rows, corrupt rows, blocks skipped for repetitive
 heads) take no part in the pipeline.
@@ -59,7 +59,7 @@ class Model(ProtocolModel):
         # a planted mistake: the speculative step releases S_b (LSE only) or writes P_b over
         # it (with P V) before it knows whether the block is redone
         self.early_p = early_p
-        self.nsb = 2 if lse_only else 3
+        self.nsb = 4 if lse_only else 3
         for name, count in [("q", 1), ("q_empty", 1), ("o_free", WARPS), ("final", 1), ("final_pv", 1)]:
             self.barrier(name, count)
         for s in range(KST):
