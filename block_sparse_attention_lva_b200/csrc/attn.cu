@@ -94,10 +94,10 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-  // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[2],
-  // s_free[2], p_full[2], o_done[2] (P*V done, per P buffer), final (Q K^T), final (P V),
-  // q_empty (an item's Q K^T done: Q may be replaced), o_free (an item's O read: P V may
-  // start the next item)
+  // barriers: q_full, k_full[KST], k_empty[KST], v_full[VST], v_empty[VST], s_full[NSB],
+  // s_free[NSB] (LSE only: S read), p_full[NSB] (P stored over S), o_done[NSB] (P*V done:
+  // the S buffer is free again), final (Q K^T), final (P V), q_empty (an item's Q K^T done:
+  // Q may be replaced), o_free (an item's O read: P V may start the next item)
   static constexpr int B_Q = 0, B_KF = 1, B_KE = B_KF + KST, B_VF = B_KE + KST, B_VE = B_VF + VST,
                        B_SF = B_VE + VST, B_SE = B_SF + NSB, B_P = B_SE + NSB, B_O = B_P + NSB,
                        B_FIN = B_O + NSB, B_FIN_PV = B_FIN + 1, B_QE = B_FIN_PV + 1, B_OF = B_QE + 1,
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
 
   // Work items: (plane, query block), plane-major with the query block fastest.  The CTA
   // takes a run of consecutive items (below).  Every role walks the same items; pipeline
-  // positions T count key blocks over all items of this CTA, so ring slots, S/P buffers and
+  // positions T count key blocks over all items of this CTA, so ring slots, S buffers and
   // their barrier phases simply continue from one item to the next, and the next item's Q
   // load and first Q K^T overlap the current item's epilogue.
   const int items = int(p.items);               // < 2^31: B*H*n_pad < 2^31 is enforced
