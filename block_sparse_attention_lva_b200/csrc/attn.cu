@@ -71,6 +71,7 @@ struct AttnParams {
   __nv_bfloat16* o_raster;         // when set: raster order [planes, n_valid, D] (o unused)
   Grid3 grid;                      // latent grid and tile of the raster order
   int64_t items;                   // (plane, query block) work items: planes * nb
+  int o_align32;                   // O rows start on 32-byte boundaries: 32-byte stores
   int gather_windows;              // 0: rows are plane-major [planes, n_pad, D]; m > 0: q, k,
                                    // v hold m windows per plane and row k of the
                                    // window-transposed order is read through a 3D map
@@ -682,14 +683,26 @@ __global__ void __launch_bounds__(kThreads, 1) bsa_fwd_kernel(
             }
           }
           if (store_o) {
+            if (p.o_align32) {
   #pragma unroll
-            for (int e4 = 0; e4 < 4; ++e4) {
-              uint32_t w4[4];
+              for (int e8 = 0; e8 < 2; ++e8) {
+                uint32_t w8[8];
   #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                w4[e] = have ? pack_bf16x2(__uint_as_float(ov[8 * e4 + 2 * e]) * inv_l,
-                                           __uint_as_float(ov[8 * e4 + 2 * e + 1]) * inv_l) : 0u;
-              reinterpret_cast<uint4*>(orow + q * 32)[e4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                for (int e = 0; e < 8; ++e)
+                  w8[e] = have ? pack_bf16x2(__uint_as_float(ov[16 * e8 + 2 * e]) * inv_l,
+                                             __uint_as_float(ov[16 * e8 + 2 * e + 1]) * inv_l) : 0u;
+                st_global_v8(orow + q * 32 + e8 * 16, w8);
+              }
+            } else {
+  #pragma unroll
+              for (int e4 = 0; e4 < 4; ++e4) {
+                uint32_t w4[4];
+  #pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  w4[e] = have ? pack_bf16x2(__uint_as_float(ov[8 * e4 + 2 * e]) * inv_l,
+                                             __uint_as_float(ov[8 * e4 + 2 * e + 1]) * inv_l) : 0u;
+                reinterpret_cast<uint4*>(orow + q * 32)[e4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+              }
             }
           }
         }
@@ -749,6 +762,7 @@ cudaError_t launch_cfg(const AttnArgs& a, cudaStream_t stream, const char** why)
   p.grid = Grid3{uint32_t(a.T), uint32_t(a.Hg), uint32_t(a.Wg), uint32_t(a.tt), uint32_t(a.th),
                  uint32_t(a.tw)};
   p.gather_windows = a.gather_windows;
+  p.o_align32 = ((reinterpret_cast<uintptr_t>(a.o_raster != nullptr ? a.o_raster : a.o) & 31) == 0) ? 1 : 0;
   p.lse = a.lse;
   p.query_src = a.query_src;
   p.src_heads = a.src_heads;

@@ -71,6 +71,35 @@ def test_against_oracle_full(B, H, n_pad, n_valid, d, bs, hm, density, seed):
     check_o_lse(o, lse, o_ref, lse_ref, f"shape {(B, H, n_pad, d, bs)}")
 
 
+
+@pytest.mark.parametrize("d,bs", [(128, 128), (64, 64)])
+def test_o_at_16_but_not_32_byte_alignment(d, bs):
+    """O rows are written with 32-byte stores when O starts on a 32-byte boundary and with
+    16-byte stores otherwise (16 bytes is the API's alignment rule): an O buffer that starts
+    16 bytes past a 32-byte boundary gets the same values, bit for bit."""
+    import block_sparse_attention_lva_b200 as lva
+    dev = require_gpu()
+    B, H, n_pad, n_valid = 1, 2, 4 * bs, 4 * bs - 3
+    q, k, v = (_rand_bf16((B, H, n_pad, d), 900 + t).to(dev) for t in range(3))
+    nb = n_pad // bs
+    masks = np.random.default_rng(9).random((1, nb, nb)) < 0.6
+    masks[0, :, 0] = True
+    rp, ci = dense_to_csr(masks)
+    row_ptr, col_idx = torch.from_numpy(rp).to(dev), torch.from_numpy(ci).to(dev)
+    scale = 1.0 / math.sqrt(d)
+    outs = []
+    for shift in (0, 8):                       # elements: 0 or 16 bytes past the allocation
+        buf = torch.full((B * H * n_pad * d + 16,), float("nan"), dtype=torch.bfloat16, device=dev)
+        o = buf[shift:shift + B * H * n_pad * d].view(B, H, n_pad, d)
+        assert (o.data_ptr() % 32 == 0) == (shift == 0)
+        lse = torch.empty((B, H, n_pad), dtype=torch.float32, device=dev)
+        lva.lva_block_sparse_attn(q, k, v, o, lse, n_valid, bs, row_ptr, col_idx, 1, scale)
+        torch.cuda.synchronize()
+        assert lva.lva_device_error() == (0, 0)
+        outs.append((o.clone(), lse.clone()))
+    assert torch.equal(outs[0][0].view(torch.int16), outs[1][0].view(torch.int16))
+    assert torch.equal(outs[0][1], outs[1][1])
+
 @pytest.mark.parametrize("d,bs", [(128, 128), (64, 64)])
 def test_all_rows_empty(d, bs):
     """An empty CSR (no entries at all): every row gives O = 0 and LSE = -inf."""
