@@ -367,9 +367,10 @@ __global__ void __launch_bounds__(kPackWarps * 32) mask_fill_packed_kernel(const
       if (row == 0) row_ptr[0] = 0;
     }
     const uint32_t* src = packed + row * wpr;
-    const int64_t nw = (nb + 31) / 32;
+    const int nw = int((nb + 31) / 32);
+    int32_t* dst = col_idx + base;
     uint32_t next = lane < nw ? __ldcs(src + lane) : 0u;
-    for (int64_t w0 = 0; w0 < nw; w0 += 32) {
+    for (int w0 = 0; w0 < nw; w0 += 32) {
       uint32_t word = next;
       next = w0 + 32 + lane < nw ? __ldcs(src + w0 + 32 + lane) : 0u;
       const int c = __popc(word);
@@ -380,7 +381,7 @@ __global__ void __launch_bounds__(kPackWarps * 32) mask_fill_packed_kernel(const
         if (lane >= o) incl += t;
       }
       const int total = __shfl_sync(0xffffffffu, incl, 31);
-      const int sh = int((reinterpret_cast<uintptr_t>(col_idx + base) >> 2) & 3);
+      const int sh = int((reinterpret_cast<uintptr_t>(dst) >> 2) & 3);
       int pos = incl - c + sh;
       const uint32_t off0 = uint32_t(lane) * 32u;          // the word's first column in the round
       while (word != 0u) {
@@ -391,23 +392,24 @@ __global__ void __launch_bounds__(kPackWarps * 32) mask_fill_packed_kernel(const
         word = rest & (rest - 1u);
       }
       __syncwarp();
-      const int32_t col0 = int32_t(w0 * 32);
-      const int end = total + sh;                          // run entries [sh, end) -> col_idx[base ...]
+      const int32_t col0 = w0 * 32;
+      const int end = total + sh;                          // run entries [sh, end) -> dst[0 ...]
       for (int c4 = lane * 4; c4 < end; c4 += 128) {
         const uint2 raw = *reinterpret_cast<const uint2*>(st + c4);
         const int32_t v0 = col0 + int32_t(raw.x & 0xffffu), v1 = col0 + int32_t(raw.x >> 16);
         const int32_t v2 = col0 + int32_t(raw.y & 0xffffu), v3 = col0 + int32_t(raw.y >> 16);
+        int32_t* o = dst + (c4 - sh);
         if (c4 >= sh && c4 + 4 <= end) {
-          *reinterpret_cast<int4*>(col_idx + base + (c4 - sh)) = make_int4(v0, v1, v2, v3);
+          *reinterpret_cast<int4*>(o) = make_int4(v0, v1, v2, v3);
         } else {
-          if (c4 >= sh && c4 < end) col_idx[base + (c4 - sh)] = v0;
-          if (c4 + 1 >= sh && c4 + 1 < end) col_idx[base + (c4 + 1 - sh)] = v1;
-          if (c4 + 2 >= sh && c4 + 2 < end) col_idx[base + (c4 + 2 - sh)] = v2;
-          if (c4 + 3 >= sh && c4 + 3 < end) col_idx[base + (c4 + 3 - sh)] = v3;
+          if (c4 >= sh && c4 < end) o[0] = v0;
+          if (c4 + 1 >= sh && c4 + 1 < end) o[1] = v1;
+          if (c4 + 2 >= sh && c4 + 2 < end) o[2] = v2;
+          if (c4 + 3 >= sh && c4 + 3 < end) o[3] = v3;
         }
       }
       __syncwarp();
-      base += total;
+      dst += total;
     }
   }
 }
